@@ -1,0 +1,177 @@
+"""Python access to the CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this package. The CUDA library does not use it, and it does not use the CUDA library.
+Arguments are numpy arrays (C-contiguous); bf16 tensors travel as uint16 bit patterns and
+E4M3 codes as uint8. Each wrapper allocates its outputs and returns them.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import LIB, build_oracle
+
+SOFTMAX = 0
+SIGMOID = 1
+OUT_BF16 = 0
+OUT_FP8_E4M3 = 1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = LIB if os.path.exists(LIB) else build_oracle()
+        _lib = ctypes.CDLL(path)
+        _declare(_lib)
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _declare(L):
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    L.tko_spec_expf.argtypes = [ctypes.c_float]
+    L.tko_spec_expf.restype = ctypes.c_float
+    L.tko_spec_sigmoidf.argtypes = [ctypes.c_float]
+    L.tko_spec_sigmoidf.restype = ctypes.c_float
+    L.tko_e4m3_encode.argtypes = [ctypes.c_float]
+    L.tko_e4m3_encode.restype = ctypes.c_uint8
+    L.tko_bf16_rne.argtypes = [ctypes.c_float]
+    L.tko_bf16_rne.restype = ctypes.c_uint16
+    for name in ("tko_spec_expf_array", "tko_spec_sigmoidf_array", "tko_e4m3_encode_array",
+                 "tko_bf16_rne_array"):
+        getattr(L, name).argtypes = [vp, vp, i64]
+        getattr(L, name).restype = None
+    L.tko_gate_topk.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    L.tko_gate_topk.restype = i32
+    L.tko_max_rows.argtypes = [i32, i32, i32, i32]
+    L.tko_max_rows.restype = i64
+    L.tko_route_map.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+    L.tko_route_map.restype = i32
+    L.tko_quantize_row_e4m3.argtypes = [vp, i32, vp, vp]
+    L.tko_quantize_row_e4m3.restype = i32
+    L.tko_expand.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+    L.tko_expand.restype = i32
+    L.tko_reduce_token.argtypes = [vp, i64, vp, vp, i32, i32, vp]
+    L.tko_reduce_token.restype = i32
+    L.tko_reduce.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp]
+    L.tko_reduce.restype = i32
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _vector(fn, x, out_dtype):
+    x = _c(x, np.float32).reshape(-1)
+    y = np.empty(x.shape, dtype=out_dtype)
+    fn(_p(x), _p(y), x.size)
+    return y
+
+
+def spec_expf(x):
+    return _vector(lib().tko_spec_expf_array, x, np.float32)
+
+
+def spec_sigmoidf(x):
+    return _vector(lib().tko_spec_sigmoidf_array, x, np.float32)
+
+
+def e4m3_encode(x):
+    return _vector(lib().tko_e4m3_encode_array, x, np.uint8)
+
+
+def bf16_rne(x):
+    return _vector(lib().tko_bf16_rne_array, x, np.uint16)
+
+
+def max_rows(T, E, k, align):
+    return int(lib().tko_max_rows(T, E, k, align))
+
+
+def gate_topk(logits, bias, k, score_fn, renormalize=True):
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    b = _c(bias, np.float32) if bias is not None else None
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float32)
+    rc = lib().tko_gate_topk(_p(logits), _p(b), T, E, k, score_fn, int(bool(renormalize)),
+                             _p(idx), _p(w))
+    if rc < 0:
+        raise ValueError(f"tko_gate_topk rejected its arguments (rc={rc})")
+    return idx, w
+
+
+def route_map(topk_idx, E, align=1):
+    topk_idx = _c(topk_idx, np.int32)
+    T, k = topk_idx.shape
+    counts = np.empty(E, dtype=np.int32)
+    offsets = np.empty(E + 1, dtype=np.int32)
+    slot_of = np.empty((T, k), dtype=np.int32)
+    token_of = np.empty(max_rows(T, E, k, align), dtype=np.int32)
+    rc = lib().tko_route_map(_p(topk_idx), T, E, k, align, _p(counts), _p(offsets), _p(slot_of),
+                             _p(token_of))
+    if rc < 0:
+        raise ValueError(f"tko_route_map rejected its arguments (rc={rc})")
+    return counts, offsets, slot_of, token_of, rc
+
+
+def quantize_row_e4m3(xrow_bits):
+    xrow_bits = _c(xrow_bits, np.uint16).reshape(-1)
+    H = xrow_bits.size
+    q = np.empty(H, dtype=np.uint8)
+    s = np.empty(H // 128, dtype=np.float32)
+    if lib().tko_quantize_row_e4m3(_p(xrow_bits), H, _p(q), _p(s)) < 0:
+        raise ValueError("tko_quantize_row_e4m3 needs H % 128 == 0")
+    return q, s
+
+
+def expand(x_bits, slot_of, offsets, E, align=1, out_dtype=OUT_BF16):
+    """Returns (out, out_scale); out has max_rows(T, E, k, align) rows, rows past offsets[E]
+    are left as zero here (the oracle never writes them)."""
+    x_bits = _c(x_bits, np.uint16)
+    slot_of = _c(slot_of, np.int32)
+    offsets = _c(offsets, np.int32)
+    T, H = x_bits.shape
+    k = slot_of.shape[1]
+    rmax = max_rows(T, E, k, align)
+    if out_dtype == OUT_BF16:
+        out = np.zeros((rmax, H), dtype=np.uint16)
+        scale = None
+    else:
+        out = np.zeros((rmax, H), dtype=np.uint8)
+        scale = np.zeros((rmax, H // 128), dtype=np.float32)
+    rc = lib().tko_expand(_p(x_bits), _p(slot_of), _p(offsets), T, E, k, H, out_dtype, _p(out),
+                          _p(scale))
+    if rc < 0:
+        raise ValueError(f"tko_expand rejected its arguments (rc={rc})")
+    return out, scale
+
+
+def reduce_token(y_bits, slot_row, w_row):
+    y_bits = _c(y_bits, np.uint16)
+    slot_row = _c(slot_row, np.int32).reshape(-1)
+    w_row = _c(w_row, np.float32).reshape(-1) if w_row is not None else None
+    H = y_bits.shape[1]
+    out = np.empty(H, dtype=np.uint16)
+    lib().tko_reduce_token(_p(y_bits), y_bits.shape[0], _p(slot_row), _p(w_row), slot_row.size, H,
+                           _p(out))
+    return out
+
+
+def reduce(y_bits, slot_of, w):
+    y_bits = _c(y_bits, np.uint16)
+    slot_of = _c(slot_of, np.int32)
+    w = _c(w, np.float32) if w is not None else None
+    T, k = slot_of.shape
+    H = y_bits.shape[1]
+    out = np.empty((T, H), dtype=np.uint16)
+    rc = lib().tko_reduce(_p(y_bits), y_bits.shape[0], _p(slot_of), _p(w), T, k, H, _p(out))
+    if rc < 0:
+        raise ValueError(f"tko_reduce rejected its arguments (rc={rc})")
+    return out
