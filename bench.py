@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE routing hot path: gate -> route map -> expand -> reduce.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tk|reference] [--workload NAME]
+
+One step = the four C-ABI calls (tk_gate_topk, tk_route_map, tk_expand, tk_reduce) over one
+synthetic batch, inputs resident in HBM. Prints ONE JSON line (rank 0). For N > 1 run it under
+torchrun: every rank routes its own batch (weak scaling, no data-path collective), time is the
+max over ranks.
+
+--impl reference times the CPU oracle (single-threaded C++) on bounded samples of the same
+workload instead; under torchrun only rank 0 works.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/s + expand/reduce HBM GB/s vs peak @T=8192,E=256,k=8,H=7168"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["tk", "reference"], default="tk")
+    p.add_argument("--workload", default="T8192_E256_k8_H7168_sigmoid_bias")
+    p.add_argument("--e2e-steps", type=int, default=None, help="end-to-end steps (default min(K, 20))")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for cpu_baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ byte accounting
+def algorithmic_bytes(wl, R=None):
+    """Bytes each call must move at minimum (read + write), per launch over the whole batch."""
+    T, E, k, H = wl.T, wl.E, wl.k, wl.H
+    R = T * k if R is None else R
+    pad_rows = R - T * k
+    gate = T * E * 4 + (E * 4 if wl.bias else 0) + T * k * 8
+    tiles = (T + 255) // 256
+    route = T * k * 4 * 3 + tiles * E * 4 * 3 + wl.max_rows * 4 + T * k * 4 * 2 + (2 * E + 1) * 4
+    if wl.out_dtype == "fp8":
+        expand = T * H * 2 + T * k * 4 + T * k * H + T * k * (H // 128) * 4
+        expand += pad_rows * (H + (H // 128) * 4)
+    else:
+        expand = T * H * 2 + T * k * 4 + T * k * H * 2 + pad_rows * H * 2
+    if wl.align > 1:
+        expand += R * 4
+    reduce = T * k * H * 2 + T * k * 8 + T * H * 2
+    return {"gate": gate, "route_map": route, "expand": expand, "reduce": reduce}
+
+
+def per_token_bytes_text(wl):
+    H, k = wl.H, wl.k
+    if wl.out_dtype == "fp8":
+        ex = f"2H + kH + 4k*H/128 + 4k = {2 * H + k * H + 4 * k * (H // 128) + 4 * k}"
+    else:
+        ex = f"2H(1+k) + 4k = {2 * H * (1 + k) + 4 * k}"
+    return {"expand": ex, "reduce": f"2H(k+1) + 8k = {2 * H * (k + 1) + 8 * k}"}
+
+
+def load_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_file, kernel_name, wl_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    source of the kernel; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[wl_name][kernel_name]
+        src = os.path.join(ROOT, "token_routing_gate_b200", "csrc", kernel_file)
+        if e.get("source_sha") != file_sha(src):
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+class ClockSampler:
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
+             0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index, period_s=0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001  (no NVML: report no clocks)
+            self.nv = None
+
+    def _reasons(self):
+        f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(self.nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return f(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons())
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self.nv is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in sorted(self.NAMES.items()) if self.reasons & b],
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def cpu_threads():
+    return 1  # the oracle is single-threaded C++
+
+
+def oracle_step(wl, lg, b, x_bits, y_bits):
+    """The whole path on the CPU oracle for one sample batch."""
+    import oracle
+    fn = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
+    idx, w = oracle.gate_topk(lg, b, wl.k, fn)
+    counts, offsets, slot_of, token_of, _ = oracle.route_map(idx, wl.E, wl.align)
+    out_dtype = oracle.OUT_FP8_E4M3 if wl.out_dtype == "fp8" else oracle.OUT_BF16
+    oracle.expand(x_bits, slot_of, offsets, wl.E, wl.align, out_dtype)
+    return oracle.reduce(y_bits, slot_of, w)
+
+
+def oracle_sample_inputs(wl, Ts, seed):
+    import numpy as np
+    import torch
+    from token_routing_gate_b200 import workloads as W
+    sw = wl.with_(T=Ts, seed=seed)
+    lg, b = W.gate_inputs(sw, "cpu")
+    x = W.activations(sw, "cpu").view(torch.int16).numpy().view(np.uint16)
+    y = W.expert_outputs(sw, "cpu").view(torch.int16).numpy().view(np.uint16)
+    return sw, lg.numpy(), (b.numpy() if b is not None else None), x, y
+
+
+def time_oracle(wl, seconds, Ts=1024):
+    from oracle.build import build_oracle
+    build_oracle()
+    sw, lg, b, x, y = oracle_sample_inputs(wl, Ts, wl.seed)
+    oracle_step(sw, lg, b, x, y)  # warm (page in)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(sw, lg, b, x, y)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n * Ts / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} runs of the full path on {Ts} tokens of {wl.name} "
+                      f"(E={wl.E}, k={wl.k}, H={wl.H}) in {el:.1f} s, single-threaded C++ oracle"}
+
+
+def run_reference(args, wl):
+    from token_routing_gate_b200 import dist
+    rank, world, _ = dist.rank_env()
+    if rank != 0:
+        return 0
+    # size each step so the whole run stays within ~2 minutes of CPU time
+    from oracle.build import build_oracle
+    build_oracle()
+    sw, lg, b, x, y = oracle_sample_inputs(wl, 128, wl.seed)
+    t0 = time.perf_counter()
+    oracle_step(sw, lg, b, x, y)
+    per_token = (time.perf_counter() - t0) / 128
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    Ts = 64
+    while Ts * 2 <= min(wl.T, 8192) and Ts * 2 * per_token <= budget:
+        Ts *= 2
+    sw, lg, b, x, y = oracle_sample_inputs(wl, Ts, wl.seed)
+    for _ in range(args.warmup):
+        oracle_step(sw, lg, b, x, y)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(sw, lg, b, x, y)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = Ts * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "E": wl.E, "k": wl.k, "H": wl.H,
+                   "score": wl.score, "bias": wl.bias, "align": wl.align, "out_dtype": wl.out_dtype,
+                   "sample_tokens_per_step": Ts},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} steps, each the full path on {Ts} tokens of "
+                                   f"{wl.name}, single-threaded C++ oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ the CUDA path
+def run_tk(args, wl):
+    import torch
+    from token_routing_gate_b200 import dist, tk
+    from token_routing_gate_b200 import workloads as W
+
+    rank, world, local_rank = dist.rank_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist.init("nccl" if world > 1 else "gloo")
+    stream = torch.cuda.current_stream(dev)
+
+    swl = wl.with_(seed=dist.shard_seed(wl.seed, rank))
+    logits, bias = W.gate_inputs(swl, dev)
+    x = W.activations(swl, dev)
+    R_max = tk.max_rows(wl.T, wl.E, wl.k, wl.align)
+    y = W.expert_outputs(swl, dev, rows=R_max)
+    # outputs, preallocated once
+    idx = torch.empty(wl.T, wl.k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.T, wl.k, dtype=torch.float32, device=dev)
+    rm = tk.route_map(idx.zero_(), wl.E, wl.align)  # allocates the route-map buffers
+    if wl.out_dtype == "fp8":
+        xe = torch.empty(R_max, wl.H, dtype=torch.uint8, device=dev)
+        xs = torch.empty(R_max, wl.H // 128, dtype=torch.float32, device=dev)
+    else:
+        xe = torch.empty(R_max, wl.H, dtype=torch.bfloat16, device=dev)
+        xs = None
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tk.gate_topk(logits, wl.k, wl.score, bias, True, idx, w, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        tk.route_map(idx, wl.E, wl.align, out=rm, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        tk.expand(x, rm, wl.E, wl.k, wl.out_dtype, out=xe, out_scale=xs, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        tk.reduce(y, rm.slot_of, w, out=out, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    launches_per_step = 1 + (3 if wl.T > 0 else 2) + 1 + (1 if wl.align > 1 else 0) + 1
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    R = int(rm.offsets[-1].item())
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for i in range(K):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    elapsed_s = start.elapsed_time(end) / 1e3
+    max_s = dist.max_over_ranks(elapsed_s, dev)
+    names = ["gate", "route_map", "expand", "reduce"]
+    k_ms = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K for j, n in enumerate(names)}
+
+    peak, peak_kind = load_peak()
+    ab = algorithmic_bytes(wl, R)
+    kernels = {n: {"us": 1e3 * k_ms[n], "bytes": ab[n], "gbs": ab[n] / (k_ms[n] / 1e3) / 1e9}
+               for n in names}
+    dom = max(("expand", "reduce"), key=lambda n: k_ms[n])
+    dom_file = {"expand": "expand.cu", "reduce": "reduce.cu"}[dom]
+    dom_kernel = {"expand": "expand_fp8_kernel" if wl.out_dtype == "fp8" else "expand_bf16_kernel",
+                  "reduce": "reduce_kernel"}[dom]
+    achieved = kernels[dom]["gbs"]
+    er_gbs = (ab["expand"] + ab["reduce"]) / ((k_ms["expand"] + k_ms["reduce"]) / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": dist.aggregate_rate(wl.T * K, world, max_s), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * max_s / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "E": wl.E, "k": wl.k, "H": wl.H,
+                   "score": wl.score, "bias": wl.bias, "align": wl.align,
+                   "out_dtype": wl.out_dtype, "tokens_per_rank": wl.T, "rows_used": R,
+                   "l2": "no flush: each step touches %.2f GB (> 126 MB L2)" % (sum(ab.values()) / 1e9),
+                   "parallelism": f"dp{world} (independent token shards, no data-path collective)"},
+        "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": ncu_traffic(dom_file, dom_kernel, wl.name),
+                     "algorithmic_bytes_per_launch": ab[dom],
+                     "per_token_bytes": per_token_bytes_text(wl)[dom]},
+        "expand_reduce": {"gbs": er_gbs, "frac": er_gbs / peak, "frac_of_8000": er_gbs / 8000.0},
+        "kernels": kernels,
+        "clocks": clocks.summary(),
+        "gpu_launches": launches_per_step * K,
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out,
+                              world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = time_oracle(wl, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.finish()
+    return 0
+
+
+def run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out, world):
+    """Same step through the public calls, with this step's inputs copied in from pinned host
+    memory and the result copied back, inside the timed region."""
+    import torch
+    from token_routing_gate_b200 import dist, tk
+
+    h_in = [t.cpu().pin_memory() for t in (logits, bias, x, y) if t is not None]
+    d_in = [t for t in (logits, bias, x, y) if t is not None]
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for d, h in zip(d_in, h_in):
+            d.copy_(h, non_blocking=True)
+        tk.gate_topk(logits, wl.k, wl.score, bias, True, idx, w, stream)
+        tk.route_map(idx, wl.E, wl.align, out=rm, stream=stream)
+        tk.expand(x, rm, wl.E, wl.k, wl.out_dtype, out=xe, out_scale=xs, stream=stream)
+        tk.reduce(y, rm.slot_of, w, out=out, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    n = args.e2e_steps if args.e2e_steps is not None else max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        e2e_step()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    max_s = dist.max_over_ranks(s.elapsed_time(e) / 1e3, dev)
+    return {"value": dist.aggregate_rate(wl.T * n, world, max_s), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "ms_per_step": 1e3 * max_s / n}
+
+
+def main():
+    args = parse_args()
+    from token_routing_gate_b200 import workloads as W
+    wl = W.BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_tk(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

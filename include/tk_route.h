@@ -1,0 +1,166 @@
+/*
+ * tk_route.h -- C ABI of libtk_route.so: the MoE gating-and-routing hot path on one B200.
+ *
+ * The path is the one the TileKernels moe/ module is described as covering ("刚刚！DeepSeek开源
+ * 高性能GPU算子库TileKernels", 147227.xyz, section "1、moe/（14个算子）"; feature list in
+ * "剛剛，DeepSeek開始頻繁更新：Tile Kernels、DeepEP V2", 機器之心, section "Tile Kernels"):
+ *   1. tk_gate_topk  -- expert scoring, top-k selection, weight renormalisation
+ *   2. tk_route_map  -- token-to-expert map: per-expert counts, segment offsets, slots
+ *   3. tk_expand     -- fused expand (dispatch): every token row copied to its k slots of an
+ *                       expert-sorted buffer, optionally quantised to FP8 E4M3 on the way
+ *   4. tk_reduce     -- fused reduce (combine): weighted sum of each token's k expert rows
+ * The pages give no signatures; arguments follow the problem statement above.
+ *
+ * Conventions for every call:
+ *  - Pointers named as device pointers must be CUDA device memory (or managed memory) that
+ *    the caller allocated and owns; the library never allocates or frees memory.
+ *  - Tensors are dense and row-major. bf16 data is passed as void* (2 bytes per element),
+ *    E4M3 data as void* (1 byte per element).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every call
+ *    only enqueues work on it and returns without synchronising the host.
+ *  - Arguments are checked on the host before anything is enqueued; a bad argument returns
+ *    TK_ERR_INVALID_ARG and enqueues nothing. tk_last_error_detail() says what was wrong.
+ *  - Data errors that only the device can see (an expert index outside [0,E), a slot outside
+ *    a buffer) never fault: the kernel skips the offending element and ORs a TK_DEVERR_* bit
+ *    into *err_flag when err_flag (a device int32, nullable) is given. The caller zeroes
+ *    *err_flag beforehand and reads it after synchronising the stream.
+ *  - Kernels launch with programmatic dependent launch enabled: each kernel may be scheduled
+ *    while the previous kernel on the stream finishes, but reads no input before that kernel
+ *    has completed.
+ */
+#ifndef TK_ROUTE_H
+#define TK_ROUTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TK_API __attribute__((visibility("default")))
+#else
+#define TK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tk_status {
+    TK_OK = 0,
+    TK_ERR_INVALID_ARG = 1, /* rejected on the host; nothing was enqueued */
+    TK_ERR_CUDA = 2         /* a CUDA runtime call or launch failed (detail has its name) */
+} tk_status;
+
+typedef enum tk_score_fn { TK_SCORE_SOFTMAX = 0, TK_SCORE_SIGMOID = 1 } tk_score_fn;
+typedef enum tk_out_dtype { TK_OUT_BF16 = 0, TK_OUT_FP8_E4M3 = 1 } tk_out_dtype;
+
+/* Bits ORed into *err_flag by the kernels. */
+#define TK_DEVERR_EXPERT_RANGE 1 /* tk_route_map: a topk_idx entry outside [0,E) (pair skipped, slot -1) */
+#define TK_DEVERR_DUP_EXPERT 2   /* tk_route_map: a token lists one expert twice (slots then overlap) */
+#define TK_DEVERR_SLOT_RANGE 4   /* tk_expand / tk_reduce: a slot outside the buffer (skipped) */
+#define TK_DEVERR_ROWS_RANGE 8   /* tk_expand: offsets[E] above the worst-case row count (clamped) */
+#define TK_DEVERR_TIMEOUT 16     /* a bounded wait inside a kernel gave up (work skipped) */
+
+/* Limits of the warp-per-token gate. */
+#define TK_MAX_EXPERTS 1024
+#define TK_MAX_TOPK 32
+
+/*
+ * Gate: expert scoring, top-k selection and weight normalisation (機器之心 "Tile Kernels"
+ * feature list: gating = top-k expert selection and scoring; routing includes weight
+ * normalisation). Selection follows the one-warp-per-token kernel sketched in the zhichai.net
+ * essay "DeepSeek 的 GPU 内核帝国", section "MoE TopK 门控": k rounds of max/argmax, ties to
+ * the lower expert index, winners written in round order.
+ *
+ *   logits  device, fp32 [T, E]
+ *   bias    device, fp32 [E] or NULL. Selection bias, sigmoid only: the key is then the fp32
+ *           value sigmoid(logit) + bias (sigmoid evaluated with the library's fixed fp32
+ *           exponential, Cody-Waite reduction + degree-7 Taylor polynomial); without a bias
+ *           the key is the logit (both score functions are increasing). NaN keys rank as -inf.
+ *   T >= 0, 1 <= E <= 1024, 1 <= k <= min(E, 32)
+ *   score_fn     TK_SCORE_SOFTMAX or TK_SCORE_SIGMOID (softmax with a bias is rejected)
+ *   renormalize  nonzero: weights are divided by their sum over the k chosen experts
+ *   topk_idx     device, int32 [T, k]: chosen experts, best first
+ *   topk_w       device, fp32 [T, k]: the unbiased scores of the chosen experts (softmax
+ *                probability or sigmoid), computed in double and rounded once to fp32;
+ *                a zero sum gives zero weights
+ */
+TK_API tk_status tk_gate_topk(const float* logits, const float* bias, int T, int E, int k, int score_fn,
+                       int renormalize, int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Worst-case number of rows of the expert-sorted buffer: T*k + E*(align-1). */
+TK_API int64_t tk_max_rows(int T, int E, int k, int align);
+
+/* Bytes of device workspace tk_route_map needs for T tokens and E experts. */
+TK_API size_t tk_route_map_workspace_bytes(int T, int E, int k);
+
+/*
+ * Token-to-expert map (機器之心 "Tile Kernels" feature list: token-to-expert mapping).
+ * Pair p = t*k + j.
+ *   topk_idx  device, int32 [T, k] (k distinct experts per token)
+ *   align     >= 1 (<= 4096): each expert's segment is padded to a multiple of align rows
+ *   counts    device, int32 [E]: pairs routed to each expert
+ *   offsets   device, int32 [E+1]: offsets[0] = 0, offsets[e+1] = offsets[e] +
+ *             ceil(counts[e]/align)*align; offsets[E] = R, the rows in use
+ *   slot_of   device, int32 [T*k]: row of pair p = offsets[e] + (number of pairs p' < p on
+ *             expert e), so each segment lists its tokens in increasing order (-1 for a pair
+ *             whose expert is out of range)
+ *   token_of  device, int32 [tk_max_rows()]: token of each row, -1 for padding rows and for
+ *             rows at and beyond R
+ *   workspace device, at least tk_route_map_workspace_bytes(T, E, k) bytes, 16-byte
+ *             aligned, no initial contents needed; not shared by calls that may overlap
+ * T*k + E*(align-1) must fit in int32.
+ */
+TK_API tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32_t* counts,
+                       int32_t* offsets, int32_t* slot_of, int32_t* token_of, void* workspace,
+                       size_t workspace_bytes, int32_t* err_flag, void* stream);
+
+/*
+ * Fused expand / dispatch (147227.xyz "moe/": fused expand; 機器之心 "性能表現": FP8 dispatch
+ * in the DeepSeek-V3 setting). Row t of x goes to rows slot_of[t*k+j], j < k, of out; padding
+ * rows (token_of == -1 below offsets[E]) are written as zeros; rows at and beyond offsets[E]
+ * are not written.
+ *   x          device, bf16 [T, H], 16-byte aligned
+ *   slot_of    device, int32 [T*k] from tk_route_map
+ *   offsets    device, int32 [E+1] from tk_route_map
+ *   token_of   device, int32 [tk_max_rows()] from tk_route_map (may be NULL when align == 1)
+ *   H          channels per row: H % 8 == 0 for bf16 output, H % 128 == 0 for E4M3 output
+ *   out_dtype  TK_OUT_BF16: out is bf16 [tk_max_rows(), H];
+ *              TK_OUT_FP8_E4M3: out is E4M3 [tk_max_rows(), H] and out_scale fp32
+ *              [tk_max_rows(), H/128]: per token and 128-channel block, scale = amax/448 and
+ *              code = E4M3(x/scale), round to nearest even, saturating at +-448 (IEEE fp32
+ *              division); a block with amax 0 gets scale 0 and codes 0. Padding rows get codes
+ *              0 and scale 0.
+ *   out        device, 16-byte aligned
+ */
+TK_API tk_status tk_expand(const void* x, const int32_t* slot_of, const int32_t* offsets,
+                    const int32_t* token_of, int T, int E, int k, int H, int align, int out_dtype,
+                    void* out, float* out_scale, int32_t* err_flag, void* stream);
+
+/*
+ * Fused reduce / combine (147227.xyz "moe/": fused reduce; 機器之心 "性能表現": BF16
+ * combine). For each token t and channel c:
+ *   acc = 0; for j = 0..k-1 in order: acc = fmaf(w[t*k+j], float(y[slot_of[t*k+j], c]), acc)
+ *   out[t, c] = bf16(acc), round to nearest even.
+ *   y        device, bf16 [y_rows, H], 16-byte aligned (expert outputs in expert-sorted rows)
+ *   slot_of  device, int32 [T*k]; a slot outside [0, y_rows) contributes nothing
+ *   w        device, fp32 [T*k] or NULL (weight 1 for every term)
+ *   H % 8 == 0
+ *   out      device, bf16 [T, H], 16-byte aligned
+ */
+TK_API tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slot_of, const float* w, int T,
+                    int k, int H, void* out, int32_t* err_flag, void* stream);
+
+/* Name of a status code (static string). */
+TK_API const char* tk_status_str(int status);
+
+/* Text describing the last non-OK status returned on the calling host thread (static
+ * thread-local buffer, valid until the next call on that thread). */
+TK_API const char* tk_last_error_detail(void);
+
+/* ABI version of this header: (major << 16) | minor. */
+TK_API int tk_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TK_ROUTE_H */

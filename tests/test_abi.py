@@ -1,0 +1,138 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point that
+include/tk_route.h declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tk_route.h")
+
+
+@pytest.fixture(scope="module")
+def tk():
+    from token_routing_gate_b200 import build
+
+    build.build()
+    from token_routing_gate_b200 import tk as mod
+
+    return mod
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^TK_API\s+[\w\s\*]+?\b(tk_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_four_steps():
+    names = _declared()
+    for n in ("tk_gate_topk", "tk_route_map", "tk_expand", "tk_reduce"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(tk):
+    L = ctypes.CDLL(tk.LIB_PATH)
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert sorted(tk.ABI_SYMBOLS) == _declared()
+
+
+def test_sizes_and_strings(tk):
+    assert tk.max_rows(8192, 256, 8, 1) == 65536
+    assert tk.max_rows(16384, 256, 8, 128) == 16384 * 8 + 256 * 127
+    assert tk.route_map_workspace_bytes(8192, 256, 8) == 32 * 256 * 4
+    assert tk.route_map_workspace_bytes(0, 16, 2) == 16 * 4
+    assert tk.lib.tk_status_str(0) == b"TK_OK"
+    assert tk.lib.tk_status_str(1) == b"TK_ERR_INVALID_ARG"
+    assert tk.lib.tk_abi_version() >> 16 == 1
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: the calls fail validation first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+@pytest.mark.parametrize("args,what", [
+    ((FAKE, None, -1, 16, 2, 0, 1, FAKE, FAKE, None), "T"),
+    ((FAKE, None, 4, 0, 1, 0, 1, FAKE, FAKE, None), "E"),
+    ((FAKE, None, 4, 2000, 2, 0, 1, FAKE, FAKE, None), "E"),
+    ((FAKE, None, 4, 16, 0, 0, 1, FAKE, FAKE, None), "k"),
+    ((FAKE, None, 4, 16, 17, 0, 1, FAKE, FAKE, None), "k"),
+    ((FAKE, None, 4, 64, 33, 0, 1, FAKE, FAKE, None), "k"),
+    ((FAKE, None, 4, 16, 2, 7, 1, FAKE, FAKE, None), "score_fn"),
+    ((FAKE, FAKE, 4, 16, 2, 0, 1, FAKE, FAKE, None), "bias"),
+    ((None, None, 4, 16, 2, 1, 1, FAKE, FAKE, None), "NULL"),
+])
+def test_gate_rejects(tk, args, what):
+    assert tk.lib.tk_gate_topk(*args) == 1
+    assert what in tk.lib.tk_last_error_detail().decode()
+
+
+def test_gate_empty_is_a_no_op(tk):
+    assert tk.lib.tk_gate_topk(None, None, 0, 16, 2, 0, 1, None, None, None) == 0
+
+
+def test_route_map_rejects(tk):
+    L = tk.lib
+    ws = tk.route_map_workspace_bytes(300, 16, 2)
+    ok = (FAKE, 300, 16, 2, 1, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None, None)
+    bad = [
+        (dict(i=4, v=0), "align"),
+        (dict(i=4, v=5000), "align"),
+        (dict(i=10, v=ws - 4), "workspace"),
+        (dict(i=9, v=MISALIGNED), "aligned"),
+        (dict(i=5, v=None), "NULL"),
+        (dict(i=8, v=None), "token_of"),
+        (dict(i=3, v=17), "k"),
+    ]
+    for change, what in bad:
+        a = list(ok)
+        a[change["i"]] = change["v"]
+        assert L.tk_route_map(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode()
+    # the worst-case row count must fit int32
+    assert L.tk_route_map(FAKE, 2**27, 1024, 32, 1, FAKE, FAKE, FAKE, FAKE, FAKE, 2**40, None, None) == 1
+
+
+def test_expand_rejects(tk):
+    L = tk.lib
+    ok = [FAKE, FAKE, FAKE, FAKE, 64, 16, 2, 256, 1, 0, FAKE, None, None, None]
+    cases = [
+        (7, 12, "H"), (7, 0, "H"), (9, 5, "out_dtype"), (8, 0, "align"), (0, MISALIGNED, "aligned"),
+        (10, MISALIGNED, "aligned"), (0, None, "NULL"), (6, 0, "k"),
+    ]
+    for i, v, what in cases:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_expand(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode()
+    a = list(ok)
+    a[9] = 1          # E4M3 output
+    a[7] = 264        # not a multiple of 128
+    a[11] = FAKE
+    assert L.tk_expand(*a) == 1 and "128" in L.tk_last_error_detail().decode()
+    a[7] = 256
+    a[11] = None      # scales missing
+    assert L.tk_expand(*a) == 1 and "out_scale" in L.tk_last_error_detail().decode()
+    a = list(ok)
+    a[8] = 128        # align > 1 needs token_of
+    a[3] = None
+    assert L.tk_expand(*a) == 1 and "token_of" in L.tk_last_error_detail().decode()
+
+
+def test_reduce_rejects(tk):
+    L = tk.lib
+    ok = [FAKE, 128, FAKE, None, 64, 2, 256, FAKE, None, None]
+    for i, v, what in [(5, 0, "k"), (5, 33, "k"), (6, 7, "H"), (1, -1, "y_rows"),
+                       (0, MISALIGNED, "aligned"), (7, MISALIGNED, "aligned"), (2, None, "NULL")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_reduce(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode()
+    assert L.tk_reduce(None, 0, None, None, 0, 2, 256, None, None, None) == 0
+
+
+def test_binding_raises_with_detail(tk):
+    with pytest.raises(tk.TkError) as ei:
+        tk._check("tk_reduce", tk.lib.tk_reduce(FAKE, 1, FAKE, None, 4, 0, 256, FAKE, None, None))
+    assert "k=0" in str(ei.value)

@@ -1,0 +1,213 @@
+// Gate: expert scoring, top-k selection and renormalisation, one warp per token.
+//
+// Selection follows the one-warp-per-token TopK kernel sketched in "DeepSeek 的 GPU 内核帝国"
+// (zhichai.net), section "MoE TopK 门控": the token's expert scores live in the warp's
+// registers, and each of k rounds takes the warp-wide maximum, resolves equal maxima to the
+// lowest expert index, records the winner and removes it. Here each lane holds experts
+// lane, lane+32, lane+64, ... (so every load of a logits row is one coalesced 128-byte line)
+// and a round is two warp reductions (redux.sync): the maximum of an order-preserving integer
+// image of the key, then the minimum expert index among the lanes holding that maximum.
+//
+// Key: the logit when no bias is given; with a bias (sigmoid scoring) the fp32 value
+// sigmoid(l) + b, where sigmoid uses a fixed fp32 exponential (Cody-Waite reduction by ln 2,
+// degree-7 Taylor polynomial, every step one IEEE fp32 operation), so the same key bits -- and
+// the same selected experts -- come out on any IEEE fp32 machine that follows the same steps.
+// Weights: the chosen experts' unbiased scores in double (library exp), renormalised over the
+// k chosen ones when asked, rounded once to fp32.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "tk_device.cuh"
+
+namespace tk {
+namespace {
+
+constexpr int kGateWarps = 8;  // tokens per CTA
+
+// e^x in fp32 for the selection key (see file comment). x is clamped to [-110, 100] first:
+// e^-110 rounds to zero and e^100 overflows, so the clamp changes no result.
+__device__ __forceinline__ float key_expf(float x) {
+    if (x != x) return x;
+    x = fminf(fmaxf(x, -110.0f), 100.0f);
+    const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));   // x * log2(e), nearest even integer
+    float r = __fmaf_rn(-n, 0x1.62e4p-1f, x);               // ln2 high part: n*hi is exact
+    r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);                  // ln2 low part
+    float p = 0x1.a01a02p-13f;                               // 1/7!
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                    // 1/6!
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);                     // 1/5!
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);                     // 1/4!
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);                     // 1/3!
+    p = __fmaf_rn(p, r, 0.5f);                               // 1/2!
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const int ni = static_cast<int>(n);
+    const int n1 = ni / 2;
+    const int n2 = ni - n1;
+    // scale by 2^n in two exact-or-single-rounding steps (|n1|, |n2| <= 80)
+    const float s1 = __int_as_float((n1 + 127) << 23);
+    const float s2 = __int_as_float((n2 + 127) << 23);
+    return __fmul_rn(__fmul_rn(p, s1), s2);
+}
+
+__device__ __forceinline__ float key_sigmoidf(float l) {
+    return __fdiv_rn(1.0f, __fadd_rn(1.0f, key_expf(-l)));
+}
+
+// Order-preserving map of an fp32 key to uint32 (larger key -> larger integer). -0 is folded
+// onto +0 and NaN onto -inf first, so float equality and integer equality agree.
+__device__ __forceinline__ uint32_t ordered_key(float key) {
+    if (key != key) key = -INFINITY;
+    key = __fadd_rn(key, 0.0f);  // -0 + 0 = +0
+    const uint32_t u = __float_as_uint(key);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One warp per token. EPL = experts held per lane (E <= 32 * EPL).
+template <int EPL>
+__global__ void __launch_bounds__(kGateWarps * 32)
+gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
+                 int k, int score_fn, int renormalize, int32_t* __restrict__ topk_idx,
+                 float* __restrict__ topk_w) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kGateWarps + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* row = logits + static_cast<int64_t>(t) * E;
+
+    float lg[EPL];      // raw logits of this lane's experts
+    uint32_t ok[EPL];   // ordered keys; 0 = removed / absent (below every real key)
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E) {
+            const float l = row[e];
+            lg[i] = l;
+            float key = l;
+            if (bias != nullptr) key = __fadd_rn(key_sigmoidf(l), bias[e]);
+            ok[i] = ordered_key(key);
+        } else {
+            lg[i] = -INFINITY;
+            ok[i] = 0u;
+        }
+    }
+    // Every real key maps above 0 (-inf maps to 0x007FFFFF), so 0 marks an absent expert
+    // (e >= E) or one already chosen, and real experts always win over absent ones.
+
+    auto local_best = [&](uint32_t& best_key, int& best_i) {
+        best_key = 0u;
+        best_i = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            if (ok[i] > best_key) { best_key = ok[i]; best_i = i; }
+        }
+    };
+    uint32_t bkey;
+    int bi;
+    local_best(bkey, bi);
+
+    int my_e = -1;        // lane j keeps the j-th winner
+    float my_l = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const uint32_t m = __reduce_max_sync(kFullMask, bkey);
+        // a lane whose best is 0 has nothing left; its candidate index is never the minimum
+        // as long as some lane holds m > 0 (always true while j < k <= E)
+        const uint32_t cand = (bkey == m) ? static_cast<uint32_t>(bi * 32 + lane) : 0xffffffffu;
+        const uint32_t win = __reduce_min_sync(kFullMask, cand);
+        const int win_lane = static_cast<int>(win & 31u);
+        const int win_i = static_cast<int>(win >> 5);
+        float wl = 0.0f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) if (i == win_i) wl = lg[i];
+        wl = __shfl_sync(kFullMask, wl, win_lane);
+        if (lane == j) { my_e = static_cast<int>(win); my_l = wl; }
+        if (lane == win_lane) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) if (i == win_i) ok[i] = 0u;
+            local_best(bkey, bi);
+        }
+    }
+
+    // ---- weights (double), lanes 0..k-1 hold the chosen experts in order
+    const float top_l = __shfl_sync(kFullMask, my_l, 0);
+    double s = 0.0;
+    bool zero_all = false;
+    if (score_fn == TK_SCORE_SIGMOID) {
+        if (lane < k) s = 1.0 / (1.0 + exp(-static_cast<double>(my_l)));
+    } else {
+        // no bias with softmax, so the first winner holds the largest logit
+        if (top_l == -INFINITY || top_l != top_l) {
+            zero_all = true;
+        } else if (lane < k) {
+            s = exp(static_cast<double>(my_l) - static_cast<double>(top_l));
+        }
+    }
+    double denom;
+    if (renormalize) {
+        double v = s;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFullMask, v, off);
+        denom = v;
+    } else if (score_fn == TK_SCORE_SOFTMAX) {
+        // full softmax denominator over all E experts
+        double z = 0.0;
+        if (!zero_all) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = i * 32 + lane;
+                if (e < E) z += exp(static_cast<double>(lg[i]) - static_cast<double>(top_l));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFullMask, z, off);
+        denom = z;
+    } else {
+        denom = 1.0;
+    }
+    if (lane < k) {
+        const int64_t o = static_cast<int64_t>(t) * k + lane;
+        topk_idx[o] = my_e;
+        topk_w[o] = (zero_all || denom == 0.0) ? 0.0f : static_cast<float>(s / denom);
+    }
+}
+
+template <int EPL>
+cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, int k, int score_fn,
+                        int renormalize, int32_t* idx, float* w, cudaStream_t s) {
+    const dim3 grid((T + kGateWarps - 1) / kGateWarps);
+    return launch_pdl(gate_topk_kernel<EPL>, grid, dim3(kGateWarps * 32), 0, s, logits, bias, T, E,
+                      k, score_fn, renormalize, idx, w);
+}
+
+}  // namespace
+}  // namespace tk
+
+extern "C" tk_status tk_gate_topk(const float* logits, const float* bias, int T, int E, int k,
+                                  int score_fn, int renormalize, int32_t* topk_idx, float* topk_w,
+                                  void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_gate_topk: T=%d must be >= 0", T);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_gate_topk: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (k < 1 || k > E || k > TK_MAX_TOPK)
+        return fail_arg("tk_gate_topk: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (score_fn != TK_SCORE_SOFTMAX && score_fn != TK_SCORE_SIGMOID)
+        return fail_arg("tk_gate_topk: unknown score_fn %d", score_fn);
+    if (score_fn == TK_SCORE_SOFTMAX && bias != nullptr)
+        return fail_arg("tk_gate_topk: a selection bias is only defined for sigmoid scoring");
+    if (T == 0) return TK_OK;
+    if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr)
+        return fail_arg("tk_gate_topk: logits, topk_idx and topk_w must not be NULL");
+    if (static_cast<int64_t>(T) * E > INT64_C(1) << 40)
+        return fail_arg("tk_gate_topk: T*E too large");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int epl = (E + 31) / 32;
+    cudaError_t err;
+    if (epl <= 1) err = launch_gate<1>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 2) err = launch_gate<2>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 4) err = launch_gate<4>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 8) err = launch_gate<8>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 16) err = launch_gate<16>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else err = launch_gate<32>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    return check_launch(err, "gate_topk_kernel");
+}

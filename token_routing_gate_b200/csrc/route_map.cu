@@ -1,0 +1,244 @@
+// Token-to-expert map: per-expert histogram -> scan for segment offsets -> stable expert-major
+// slots (機器之心 "剛剛，DeepSeek開始頻繁更新", section "Tile Kernels": token-to-expert
+// mapping is one of the MoE routing ops).
+//
+// The pairs p = t*k + j are cut into tiles of kTileTokens tokens. Three short kernels:
+//   count   : one CTA per tile counts its pairs per expert in shared memory (warp-aggregated
+//             atomics; counts do not depend on their order) and writes a row of the
+//             [tiles x E] count matrix; the grid also fills token_of with -1.
+//   scan    : one CTA turns each column of the matrix into exclusive per-tile prefixes, sums
+//             the column into counts[e], rounds it up to the alignment and scans over experts
+//             for offsets[].
+//   scatter : one CTA per tile marks, per expert, which of its tokens chose that expert in a
+//             shared-memory bitmap; a pair's rank inside the tile is the population count of
+//             the bits below its token. slot = offsets[e] + tile prefix[e] + rank -- the same
+//             number a sequential pass in p order hands out, with no dependence on thread
+//             timing.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tk_device.cuh"
+
+namespace tk {
+namespace {
+
+constexpr int kTileTokens = 256;               // tokens per tile
+constexpr int kTileWords = kTileTokens / 32;   // bitmap words per expert
+constexpr int kRouteThreads = 256;
+constexpr int kScanThreads = 1024;
+
+inline int num_tiles(int T) { return (T + kTileTokens - 1) / kTileTokens; }
+
+__global__ void __launch_bounds__(kRouteThreads)
+route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                   int32_t* __restrict__ tile_counts, int32_t* __restrict__ token_of,
+                   int64_t rmax, int32_t* err_flag) {
+    extern __shared__ int32_t cnt[];  // [E]
+    pdl_wait();
+    pdl_trigger();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    // every row starts as "no token"; the scatter kernel fills the real rows afterwards
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < rmax;
+         r += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        token_of[r] = -1;
+    __syncthreads();
+    const int tile = blockIdx.x;
+    const int64_t p0 = static_cast<int64_t>(tile) * kTileTokens * k;
+    const int64_t p1 = min(static_cast<int64_t>(T), static_cast<int64_t>(tile + 1) * kTileTokens) * k;
+    // all 32 lanes of a warp run the same number of iterations, so __match_any_sync sees a full
+    // warp; lanes past the tile carry the sentinel -1
+    for (int64_t base = p0; base < p1; base += blockDim.x) {
+        const int64_t p = base + threadIdx.x;
+        int e = -1;
+        if (p < p1) {
+            e = topk_idx[p];
+            if (e < 0 || e >= E) {
+                flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
+                e = -1;
+            }
+        }
+        const unsigned peers = __match_any_sync(kFullMask, e);
+        const int lane = threadIdx.x & 31;
+        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt[e], __popc(peers));
+    }
+    __syncthreads();
+    if (p0 < p1 || tile == 0) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            tile_counts[static_cast<int64_t>(tile) * E + e] = cnt[e];
+    }
+}
+
+// Single CTA. Column e of tile_counts becomes exclusive per-tile prefixes (in place).
+__global__ void __launch_bounds__(kScanThreads)
+route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align,
+                  int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+    __shared__ int32_t warp_tot[kScanThreads / 32];
+    __shared__ int32_t carry;
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    // experts in chunks of blockDim.x; each thread owns one expert of the chunk
+    for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+        const int e = e0 + threadIdx.x;
+        int32_t padded = 0;
+        if (e < E) {
+            int32_t run = 0;
+            int c = 0;
+            for (; c + 4 <= tiles; c += 4) {
+                const int32_t v0 = tile_counts[static_cast<int64_t>(c) * E + e];
+                const int32_t v1 = tile_counts[static_cast<int64_t>(c + 1) * E + e];
+                const int32_t v2 = tile_counts[static_cast<int64_t>(c + 2) * E + e];
+                const int32_t v3 = tile_counts[static_cast<int64_t>(c + 3) * E + e];
+                tile_counts[static_cast<int64_t>(c) * E + e] = run;
+                tile_counts[static_cast<int64_t>(c + 1) * E + e] = run + v0;
+                tile_counts[static_cast<int64_t>(c + 2) * E + e] = run + v0 + v1;
+                tile_counts[static_cast<int64_t>(c + 3) * E + e] = run + v0 + v1 + v2;
+                run += v0 + v1 + v2 + v3;
+            }
+            for (; c < tiles; ++c) {
+                const int32_t v = tile_counts[static_cast<int64_t>(c) * E + e];
+                tile_counts[static_cast<int64_t>(c) * E + e] = run;
+                run += v;
+            }
+            counts[e] = run;
+            padded = (run + align - 1) / align * align;
+        }
+        // block-wide exclusive scan of padded over this chunk of experts
+        int32_t incl = padded;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t v = __shfl_up_sync(kFullMask, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int nw = blockDim.x / 32;
+            int32_t v = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int32_t u = __shfl_up_sync(kFullMask, v, off);
+                if (lane >= off) v += u;
+            }
+            if (lane < nw) warp_tot[lane] = v;  // inclusive over warps
+        }
+        __syncthreads();
+        const int32_t warp_excl = warp > 0 ? warp_tot[warp - 1] : 0;
+        const int32_t excl = carry + warp_excl + incl - padded;
+        if (e < E) offsets[e] = excl;
+        const int32_t chunk_total = warp_tot[blockDim.x / 32 - 1];
+        __syncthreads();
+        if (threadIdx.x == 0) carry += chunk_total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) offsets[E] = carry;
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                     const int32_t* __restrict__ tile_prefix, const int32_t* __restrict__ offsets,
+                     int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
+                     int32_t* err_flag) {
+    extern __shared__ uint32_t smem[];
+    uint32_t* bitmap = smem;                                          // [E][kTileWords]
+    int32_t* base = reinterpret_cast<int32_t*>(smem + E * kTileWords);  // [E]
+    pdl_wait();
+    pdl_trigger();
+    const int tile = blockIdx.x;
+    const int t0 = tile * kTileTokens;
+    const int64_t p0 = static_cast<int64_t>(t0) * k;
+    const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
+    for (int i = threadIdx.x; i < E * kTileWords; i += blockDim.x) bitmap[i] = 0u;
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(tile) * E + e];
+    __syncthreads();
+    for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+        const int e = topk_idx[p];
+        if (e < 0 || e >= E) continue;  // flagged by the count kernel
+        const int tl = static_cast<int>(p / k) - t0;
+        const uint32_t bit = 1u << (tl & 31);
+        const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
+        if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
+    }
+    __syncthreads();
+    for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+        const int e = topk_idx[p];
+        if (e < 0 || e >= E) {
+            slot_of[p] = -1;
+            continue;
+        }
+        const int t = static_cast<int>(p / k);
+        const int tl = t - t0;
+        const uint32_t* bm = bitmap + e * kTileWords;
+        int rank = __popc(bm[tl >> 5] & ((1u << (tl & 31)) - 1u));
+        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bm[w]);
+        const int32_t slot = base[e] + rank;
+        slot_of[p] = slot;
+        token_of[slot] = t;
+    }
+}
+
+}  // namespace
+
+size_t route_map_workspace_bytes_impl(int T, int E) {
+    const int tiles = num_tiles(T) > 0 ? num_tiles(T) : 1;
+    return static_cast<size_t>(tiles) * static_cast<size_t>(E) * sizeof(int32_t);
+}
+
+}  // namespace tk
+
+extern "C" int64_t tk_max_rows(int T, int E, int k, int align) {
+    return static_cast<int64_t>(T) * k + static_cast<int64_t>(E) * (align - 1);
+}
+
+extern "C" size_t tk_route_map_workspace_bytes(int T, int E, int k) {
+    (void)k;
+    if (T < 0 || E < 1) return 0;
+    return tk::route_map_workspace_bytes_impl(T, E);
+}
+
+extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int align,
+                                  int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                                  int32_t* token_of, void* workspace, size_t workspace_bytes,
+                                  int32_t* err_flag, void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_route_map: T=%d must be >= 0", T);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_route_map: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (k < 1 || k > E || k > TK_MAX_TOPK)
+        return fail_arg("tk_route_map: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (align < 1 || align > 4096) return fail_arg("tk_route_map: align=%d outside [1, 4096]", align);
+    const int64_t rmax = tk_max_rows(T, E, k, align);
+    if (rmax > INT32_MAX) return fail_arg("tk_route_map: T*k + E*(align-1) = %lld exceeds int32", (long long)rmax);
+    if (counts == nullptr || offsets == nullptr || workspace == nullptr)
+        return fail_arg("tk_route_map: counts, offsets and workspace must not be NULL");
+    if (T > 0 && (topk_idx == nullptr || slot_of == nullptr))
+        return fail_arg("tk_route_map: topk_idx and slot_of must not be NULL");
+    if (rmax > 0 && token_of == nullptr) return fail_arg("tk_route_map: token_of must not be NULL");
+    const size_t need = route_map_workspace_bytes_impl(T, E);
+    if (workspace_bytes < need)
+        return fail_arg("tk_route_map: workspace holds %zu bytes, needs %zu", workspace_bytes, need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+        return fail_arg("tk_route_map: workspace must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* tile_counts = static_cast<int32_t*>(workspace);
+    const int tiles = num_tiles(T);
+    const int count_grid = tiles > 0 ? tiles : 1;
+    cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
+                                 static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
+                                 tile_counts, token_of, rmax, err_flag);
+    if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
+    err = launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tile_counts, tiles, E,
+                     align, counts, offsets);
+    if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
+    if (tiles > 0) {
+        const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
+        err = launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
+                         T, E, k, static_cast<const int32_t*>(tile_counts),
+                         static_cast<const int32_t*>(offsets), slot_of, token_of, err_flag);
+        if (err != cudaSuccess) return check_launch(err, "route_scatter_kernel");
+    }
+    return TK_OK;
+}

@@ -1,0 +1,160 @@
+"""Thin Python binding of libtk_route.so (C ABI in include/tk_route.h).
+
+Argument marshalling only: torch tensors supply device memory and the current CUDA stream,
+every step runs in the library's kernels. The names follow the C entry points without the
+``tk_`` prefix. Missing outputs are allocated with torch (caching allocator) before the call;
+pass preallocated tensors to keep allocation out of a timed loop. There is no fallback: if the
+library is not built, importing this module raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtk_route.so")
+
+SCORE = {"softmax": 0, "sigmoid": 1}
+OUT_DTYPE = {"bf16": 0, "fp8": 1}
+
+DEVERR_EXPERT_RANGE = 1
+DEVERR_DUP_EXPERT = 2
+DEVERR_SLOT_RANGE = 4
+DEVERR_ROWS_RANGE = 8
+DEVERR_TIMEOUT = 16
+
+# every C entry point declared in include/tk_route.h
+ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
+               "tk_expand", "tk_reduce", "tk_status_str", "tk_last_error_detail",
+               "tk_abi_version")
+
+
+class TkError(RuntimeError):
+    def __init__(self, fn, status, detail):
+        super().__init__(f"{fn} failed: {status} -- {detail}")
+        self.status = status
+        self.detail = detail
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is not built; run `python -m token_routing_gate_b200.build` "
+            "(the CUDA library is required, there is no CPU path)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    L.tk_gate_topk.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.tk_gate_topk.restype = i32
+    L.tk_max_rows.argtypes = [i32, i32, i32, i32]
+    L.tk_max_rows.restype = i64
+    L.tk_route_map_workspace_bytes.argtypes = [i32, i32, i32]
+    L.tk_route_map_workspace_bytes.restype = sz
+    L.tk_route_map.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.tk_route_map.restype = i32
+    L.tk_expand.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+    L.tk_expand.restype = i32
+    L.tk_reduce.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp, vp, vp]
+    L.tk_reduce.restype = i32
+    L.tk_status_str.argtypes = [i32]
+    L.tk_status_str.restype = ctypes.c_char_p
+    L.tk_last_error_detail.argtypes = []
+    L.tk_last_error_detail.restype = ctypes.c_char_p
+    L.tk_abi_version.argtypes = []
+    L.tk_abi_version.restype = i32
+    return L
+
+
+lib = _load()
+
+
+def _check(fn, status):
+    if status != 0:
+        raise TkError(fn, lib.tk_status_str(status).decode(), lib.tk_last_error_detail().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libtk_route must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def max_rows(T, E, k, align=1):
+    return int(lib.tk_max_rows(T, E, k, align))
+
+
+def route_map_workspace_bytes(T, E, k):
+    return int(lib.tk_route_map_workspace_bytes(T, E, k))
+
+
+def gate_topk(logits, k, score="sigmoid", bias=None, renormalize=True, topk_idx=None, topk_w=None,
+              stream=None):
+    """logits fp32 [T,E] -> (topk_idx int32 [T,k], topk_w fp32 [T,k])."""
+    T, E = logits.shape
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
+    _check("tk_gate_topk", lib.tk_gate_topk(_ptr(logits), _ptr(bias), T, E, k, SCORE[score],
+                                            int(bool(renormalize)), _ptr(topk_idx), _ptr(topk_w),
+                                            _stream(stream)))
+    return topk_idx, topk_w
+
+
+class RouteMap:
+    """Outputs of route_map: counts [E], offsets [E+1], slot_of [T,k], token_of [max_rows]."""
+
+    def __init__(self, counts, offsets, slot_of, token_of, workspace, align):
+        self.counts, self.offsets, self.slot_of, self.token_of = counts, offsets, slot_of, token_of
+        self.workspace = workspace
+        self.align = align
+
+
+def route_map(topk_idx, E, align=1, out=None, err_flag=None, stream=None):
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if out is None:
+        ws = max(route_map_workspace_bytes(T, E, k), 16)
+        out = RouteMap(torch.empty(E, dtype=torch.int32, device=dev),
+                       torch.empty(E + 1, dtype=torch.int32, device=dev),
+                       torch.empty(T, k, dtype=torch.int32, device=dev),
+                       torch.empty(max(max_rows(T, E, k, align), 1), dtype=torch.int32, device=dev),
+                       torch.empty((ws + 15) // 16, 16, dtype=torch.uint8, device=dev), align)
+    _check("tk_route_map", lib.tk_route_map(
+        _ptr(topk_idx), T, E, k, align, _ptr(out.counts), _ptr(out.offsets), _ptr(out.slot_of),
+        _ptr(out.token_of), _ptr(out.workspace), out.workspace.numel(), _ptr(err_flag),
+        _stream(stream)))
+    return out
+
+
+def expand(x, rm, E, k, out_dtype="bf16", out=None, out_scale=None, err_flag=None, stream=None):
+    """x bf16 [T,H] -> out [max_rows, H] (bf16, or E4M3 as uint8 with fp32 scales [max_rows, H/128])."""
+    T, H = x.shape
+    R = max(max_rows(T, E, k, rm.align), 1)
+    if out is None:
+        out = torch.empty(R, H, dtype=torch.bfloat16 if out_dtype == "bf16" else torch.uint8,
+                          device=x.device)
+    if out_dtype == "fp8" and out_scale is None:
+        out_scale = torch.empty(R, H // 128, dtype=torch.float32, device=x.device)
+    _check("tk_expand", lib.tk_expand(
+        _ptr(x), _ptr(rm.slot_of), _ptr(rm.offsets), _ptr(rm.token_of), T, E, k, H, rm.align,
+        OUT_DTYPE[out_dtype], _ptr(out), _ptr(out_scale), _ptr(err_flag), _stream(stream)))
+    return (out, out_scale) if out_dtype == "fp8" else out
+
+
+def reduce(y, slot_of, w=None, out=None, err_flag=None, stream=None):
+    """y bf16 [rows,H], slot_of int32 [T,k], w fp32 [T,k] or None -> out bf16 [T,H]."""
+    T, k = slot_of.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device)
+    _check("tk_reduce", lib.tk_reduce(_ptr(y), y.shape[0], _ptr(slot_of), _ptr(w), T, k, H,
+                                      _ptr(out), _ptr(err_flag), _stream(stream)))
+    return out
