@@ -32,10 +32,12 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["tk", "reference"], default="tk")
     p.add_argument("--workload", default="T8192_E256_k8_H7168_sigmoid_bias")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override T of the workload (smaller cases for profiling)")
     p.add_argument("--e2e-steps", type=int, default=None, help="end-to-end steps (default min(K, 20))")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for cpu_baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -108,7 +110,7 @@ class ClockSampler:
     NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
              0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
-    def __init__(self, index, period_s=0.01):
+    def __init__(self, index, period_s=0.002):
         self.index, self.period = index, period_s
         self.samples, self.reasons = [], 0
         self.max_mhz = None
@@ -256,7 +258,7 @@ def run_tk(args, wl):
     dist.init("nccl" if world > 1 else "gloo")
     stream = torch.cuda.current_stream(dev)
 
-    swl = wl.with_(seed=dist.shard_seed(wl.seed, rank))
+    swl = wl.with_(seed=dist.shard_seed(wl.seed, rank), param_seed=wl.seed)
     logits, bias = W.gate_inputs(swl, dev)
     x = W.activations(swl, dev)
     R_max = tk.max_rows(wl.T, wl.E, wl.k, wl.align)
@@ -397,6 +399,8 @@ def main():
     args = parse_args()
     from token_routing_gate_b200 import workloads as W
     wl = W.BY_NAME[args.workload]
+    if args.tokens is not None:
+        wl = wl.with_(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_tk(args, wl)

@@ -63,6 +63,34 @@ __device__ __forceinline__ uint32_t ordered_key(float key) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Packs an ordered key and an expert index into one 64-bit value whose unsigned order is
+// (key descending, index ascending): the high word is the key's image, the low word ~e.
+__device__ __forceinline__ uint64_t pack_key(uint32_t ord, int e) {
+    return (static_cast<uint64_t>(ord) << 32) | static_cast<uint32_t>(~e);
+}
+
+// Sorts a lane's EPL packed values in descending order (bitonic network, fully unrolled).
+template <int EPL>
+__device__ __forceinline__ void sort_desc(uint64_t (&v)[EPL]) {
+#pragma unroll
+    for (int size = 2; size <= EPL; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int l = i ^ stride;
+                if (l > i) {
+                    const bool desc = (i & size) == 0;
+                    const uint64_t a = v[i], b = v[l];
+                    const bool swap = desc ? (a < b) : (a > b);
+                    v[i] = swap ? b : a;
+                    v[l] = swap ? a : b;
+                }
+            }
+        }
+    }
+}
+
 // One warp per token. EPL = experts held per lane (E <= 32 * EPL).
 template <int EPL>
 __global__ void __launch_bounds__(kGateWarps * 32)
@@ -76,58 +104,35 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
     if (t >= T) return;
     const float* row = logits + static_cast<int64_t>(t) * E;
 
-    float lg[EPL];      // raw logits of this lane's experts
-    uint32_t ok[EPL];   // ordered keys; 0 = removed / absent (below every real key)
+    // Every real key maps above 0 (-inf maps to 0x007FFFFF), so 0 marks an absent expert
+    // (e >= E) or one already chosen, and real experts always win over absent ones.
+    uint64_t v[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = i * 32 + lane;
+        v[i] = 0;
         if (e < E) {
             const float l = row[e];
-            lg[i] = l;
-            float key = l;
-            if (bias != nullptr) key = __fadd_rn(key_sigmoidf(l), bias[e]);
-            ok[i] = ordered_key(key);
-        } else {
-            lg[i] = -INFINITY;
-            ok[i] = 0u;
+            const float key = bias != nullptr ? __fadd_rn(key_sigmoidf(l), bias[e]) : l;
+            v[i] = pack_key(ordered_key(key), e);
         }
     }
-    // Every real key maps above 0 (-inf maps to 0x007FFFFF), so 0 marks an absent expert
-    // (e >= E) or one already chosen, and real experts always win over absent ones.
+    if (EPL > 1) sort_desc<EPL>(v);
 
-    auto local_best = [&](uint32_t& best_key, int& best_i) {
-        best_key = 0u;
-        best_i = 0;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            if (ok[i] > best_key) { best_key = ok[i]; best_i = i; }
-        }
-    };
-    uint32_t bkey;
-    int bi;
-    local_best(bkey, bi);
-
-    int my_e = -1;        // lane j keeps the j-th winner
-    float my_l = 0.0f;
+    int my_e = 0;  // lane j keeps the j-th winner
     for (int j = 0; j < k; ++j) {
-        const uint32_t m = __reduce_max_sync(kFullMask, bkey);
-        // a lane whose best is 0 has nothing left; its candidate index is never the minimum
-        // as long as some lane holds m > 0 (always true while j < k <= E)
-        const uint32_t cand = (bkey == m) ? static_cast<uint32_t>(bi * 32 + lane) : 0xffffffffu;
-        const uint32_t win = __reduce_min_sync(kFullMask, cand);
-        const int win_lane = static_cast<int>(win & 31u);
-        const int win_i = static_cast<int>(win >> 5);
-        float wl = 0.0f;
+        const uint32_t hi = static_cast<uint32_t>(v[0] >> 32);
+        const uint32_t m = __reduce_max_sync(kFullMask, hi);
+        const uint32_t lo = static_cast<uint32_t>(v[0]);
+        const uint32_t win = __reduce_max_sync(kFullMask, hi == m ? lo : 0u);  // ~e: lower e wins
+        if (lane == j) my_e = static_cast<int>(~win);
+        if (hi == m && lo == win) {  // the one lane holding the winner drops it
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) if (i == win_i) wl = lg[i];
-        wl = __shfl_sync(kFullMask, wl, win_lane);
-        if (lane == j) { my_e = static_cast<int>(win); my_l = wl; }
-        if (lane == win_lane) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) if (i == win_i) ok[i] = 0u;
-            local_best(bkey, bi);
+            for (int i = 0; i + 1 < EPL; ++i) v[i] = v[i + 1];
+            v[EPL - 1] = 0;
         }
     }
+    const float my_l = lane < k ? row[my_e] : 0.0f;
 
     // ---- weights (double), lanes 0..k-1 hold the chosen experts in order
     const float top_l = __shfl_sync(kFullMask, my_l, 0);
@@ -156,7 +161,7 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = i * 32 + lane;
-                if (e < E) z += exp(static_cast<double>(lg[i]) - static_cast<double>(top_l));
+                if (e < E) z += exp(static_cast<double>(row[e]) - static_cast<double>(top_l));
             }
         }
 #pragma unroll

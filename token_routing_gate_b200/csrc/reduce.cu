@@ -2,12 +2,21 @@
 // in slot order j = 0..k-1, one fmaf per term (147227.xyz "刚刚！DeepSeek开源高性能GPU算子库
 // TileKernels", section "moe/": fused reduce; BF16 combine in 機器之心 "性能表現").
 //
-// Pure bandwidth: k scattered 2H-byte rows read, one 2H-byte row written per token. Work unit =
-// one warp x (token, 64 consecutive 8-channel vectors); each lane owns two vectors 32 apart,
-// so every load instruction of the warp covers 512 contiguous bytes of one row. A lane issues
-// all its loads for up to 8 rows (16 x 16 bytes in flight) before the first FMA, which keeps
-// enough bytes in flight per SM to cover HBM latency. The grid is persistent (a few CTAs per
-// SM, sized by the occupancy calculator) and strides over units.
+// Pure bandwidth: per token, k scattered 2H-byte rows read and one 2H-byte row written. The
+// loads go through the bulk-copy (TMA) engine so that the bytes in flight do not depend on
+// registers: a unit of work is (token t, 1024-channel chunk c). Each CTA is warp-specialised:
+//   warp 0      producer: lanes j < k read slot j and weight j of the unit, park the weights in
+//               the stage's shared-memory header, and issue one 1-D bulk load per valid row
+//               chunk (2 KB each) into the stage, completing on the stage's "full" mbarrier
+//               (transaction count = bytes issued).
+//   warps 1..4  consumers: wait "full", each thread combines one 8-channel vector of the unit
+//               across the k row chunks (16-byte shared loads, fmaf in slot order), writes 16
+//               bytes of bf16 output, then the warp arrives on the stage's "empty" mbarrier.
+// The ring has S stages with S*k*2 KB <= 32 KB (two at k = 8), so an SM holds about six CTAs and
+// up to ~190 KB of loads in flight. A measured sweep on B200 (ring depth, chunk width, consumer
+// warps) put this shape at the HBM copy roofline; deeper rings with fewer CTAs per SM were up to
+// 30% slower. The grid is persistent (SM count x CTAs per SM) and CTAs stride over units. Every wait is bounded (1 s); a timeout flags TK_DEVERR_TIMEOUT and ends the
+// CTA's loop.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -17,10 +26,28 @@
 namespace tk {
 namespace {
 
-constexpr int kRedThreads = 256;
-constexpr int kRedWarps = kRedThreads / 32;
-constexpr int kU = 2;    // 8-channel vectors per lane per unit
-constexpr int kKC = 8;   // rows whose loads are issued together
+#ifndef TK_REDUCE_CONSUMER_WARPS
+#define TK_REDUCE_CONSUMER_WARPS 4
+#endif
+#ifndef TK_REDUCE_VECS_PER_THREAD
+#define TK_REDUCE_VECS_PER_THREAD 1
+#endif
+#ifndef TK_REDUCE_STAGE_KB
+#define TK_REDUCE_STAGE_KB 32
+#endif
+
+constexpr int kConsumerWarps = TK_REDUCE_CONSUMER_WARPS;
+constexpr int kVecs = TK_REDUCE_VECS_PER_THREAD;        // 8-channel vectors per consumer thread
+constexpr int kRedThreads = 32 * (1 + kConsumerWarps);
+constexpr int kChunkCh = 8 * 32 * kConsumerWarps * kVecs;  // channels per unit
+constexpr int kChunkBytes = kChunkCh * 2;                  // bf16 bytes of one row chunk
+constexpr int kStageBudget = TK_REDUCE_STAGE_KB * 1024;    // shared bytes of row data per CTA
+constexpr int kMaxStages = 8;
+
+struct StageMeta {
+    float w[TK_MAX_TOPK];
+    int32_t valid[TK_MAX_TOPK];
+};
 
 __device__ __forceinline__ float lo_bf16(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
@@ -31,95 +58,171 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
+int stages_for(int k) {
+#ifdef TK_REDUCE_STAGES
+    (void)k;
+    return TK_REDUCE_STAGES;
+#endif
+    int s = kStageBudget / (k * kChunkBytes);
+    if (s < 1) s = 1;
+    if (s > kMaxStages) s = kMaxStages;
+    return s;
+}
+
+size_t smem_bytes(int k, int S) {
+    return static_cast<size_t>(S) * k * kChunkBytes + static_cast<size_t>(S) * sizeof(StageMeta) +
+           static_cast<size_t>(2 * S) * sizeof(uint64_t);
+}
+
 __global__ void __launch_bounds__(kRedThreads)
 reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __restrict__ slot_of,
-              const float* __restrict__ w, int T, int k, int H, uint8_t* __restrict__ out,
+              const float* __restrict__ w, int T, int k, int H, int S, uint8_t* __restrict__ out,
               int32_t* err_flag) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    const int stage_bytes = k * kChunkBytes;
+    uint8_t* data = sm;
+    StageMeta* meta = reinterpret_cast<StageMeta*>(sm + static_cast<size_t>(S) * stage_bytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(meta + S);
+    uint64_t* empty = full + S;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
     pdl_wait();
     pdl_trigger();
-    const int lane = threadIdx.x & 31;
-    const int V = H / 8;                                 // 16-byte vectors per row
-    const int units_per_token = (V + 32 * kU - 1) / (32 * kU);
-    const int64_t total_units = static_cast<int64_t>(T) * units_per_token;
-    const int64_t row_bytes = static_cast<int64_t>(H) * 2;
-    for (int64_t unit = static_cast<int64_t>(blockIdx.x) * kRedWarps + (threadIdx.x >> 5);
-         unit < total_units; unit += static_cast<int64_t>(gridDim.x) * kRedWarps) {
-        const int64_t t = unit / units_per_token;
-        const int vbase = static_cast<int>(unit - t * units_per_token) * (32 * kU);
-        int64_t my_slot = -1;
-        float my_w = 1.0f;
-        if (lane < k) {
-            const int64_t s = slot_of[t * k + lane];
-            if (s >= 0 && s < y_rows) my_slot = s;
-            else if (s != -1) flag_error(err_flag, TK_DEVERR_SLOT_RANGE);
-            if (w != nullptr) my_w = w[t * k + lane];
-        }
-        float acc[kU][8];
-#pragma unroll
-        for (int u = 0; u < kU; ++u)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[u][e] = 0.0f;
-        bool vec_ok[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) vec_ok[u] = vbase + u * 32 + lane < V;
 
-        for (int j0 = 0; j0 < k; j0 += kKC) {
-            uint4 v[kKC][kU];
-            int64_t sl[kKC];
-#pragma unroll
-            for (int jj = 0; jj < kKC; ++jj) {
-                sl[jj] = __shfl_sync(kFullMask, my_slot, (j0 + jj) & 31);
-                const bool live = (j0 + jj < k) && sl[jj] >= 0;
-#pragma unroll
-                for (int u = 0; u < kU; ++u) {
-                    v[jj][u] = make_uint4(0u, 0u, 0u, 0u);
-                    if (live && vec_ok[u])
-                        v[jj][u] = ld_stream_v4(y + sl[jj] * row_bytes +
-                                                static_cast<int64_t>(vbase + u * 32 + lane) * 16);
-                }
-            }
-#pragma unroll
-            for (int jj = 0; jj < kKC; ++jj) {
-                const float wj = __shfl_sync(kFullMask, my_w, (j0 + jj) & 31);
-                if (j0 + jj < k && sl[jj] >= 0) {
-#pragma unroll
-                    for (int u = 0; u < kU; ++u) {
-                        const uint4 q = v[jj][u];
-                        acc[u][0] = __fmaf_rn(wj, lo_bf16(q.x), acc[u][0]);
-                        acc[u][1] = __fmaf_rn(wj, hi_bf16(q.x), acc[u][1]);
-                        acc[u][2] = __fmaf_rn(wj, lo_bf16(q.y), acc[u][2]);
-                        acc[u][3] = __fmaf_rn(wj, hi_bf16(q.y), acc[u][3]);
-                        acc[u][4] = __fmaf_rn(wj, lo_bf16(q.z), acc[u][4]);
-                        acc[u][5] = __fmaf_rn(wj, hi_bf16(q.z), acc[u][5]);
-                        acc[u][6] = __fmaf_rn(wj, lo_bf16(q.w), acc[u][6]);
-                        acc[u][7] = __fmaf_rn(wj, hi_bf16(q.w), acc[u][7]);
-                    }
-                }
-            }
+    const int chunks = (H + kChunkCh - 1) / kChunkCh;
+    const int64_t units = static_cast<int64_t>(T) * chunks;
+    const int64_t row_bytes = static_cast<int64_t>(H) * 2;
+
+    if (warp == 0) {
+        // ---------------- producer (slots and weights of the next unit are fetched while the
+        // current unit waits for a free stage)
+        int64_t u = blockIdx.x;
+        int64_t nxt_sl = -1;
+        float nxt_w = 1.0f;
+        if (lane < k && u < units) {
+            const int64_t t = u / chunks;
+            nxt_sl = slot_of[t * k + lane];
+            if (w != nullptr) nxt_w = w[t * k + lane];
         }
+        for (int it = 0; u < units; u += gridDim.x, ++it) {
+            const int s = it % S;
+            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+            const int64_t t = u / chunks;
+            const int ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
+            const uint32_t bytes = static_cast<uint32_t>(min(kChunkCh, H - ch0)) * 2u;
+            const int64_t raw = nxt_sl;
+            const float wl = nxt_w;
+            const int64_t un = u + gridDim.x;
+            if (lane < k && un < units) {
+                const int64_t tn = un / chunks;
+                nxt_sl = slot_of[tn * k + lane];
+                if (w != nullptr) nxt_w = w[tn * k + lane];
+            }
+            int64_t sl = -1;
+            if (lane < k) {
+                if (raw >= 0 && raw < y_rows) sl = raw;
+                else if (raw != -1) flag_error(err_flag, TK_DEVERR_SLOT_RANGE);
+            }
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(&empty[s], ph ^ 1u) ? 1 : 0;
+            ok = __shfl_sync(kFullMask, ok, 0);
+            if (!ok) {
+                if (lane == 0) flag_error(err_flag, TK_DEVERR_TIMEOUT);
+                break;
+            }
+            if (lane < k) {
+                meta[s].w[lane] = wl;
+                meta[s].valid[lane] = sl >= 0 ? 1 : 0;
+            }
+            const unsigned vmask = __ballot_sync(kFullMask, sl >= 0);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(vmask)) * bytes);
+            __syncwarp();
+            if (sl >= 0)
+                bulk_load(data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * kChunkBytes,
+                          y + sl * row_bytes + static_cast<int64_t>(ch0) * 2, bytes, &full[s]);
+        }
+    } else {
+        // ---------------- consumers
+        const int ct = threadIdx.x - 32;  // 0 .. 32*kConsumerWarps-1
+        int it = 0;
+        for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+            const int s = it % S;
+            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+            if (!mbar_wait_bounded(&full[s], ph)) {
+                flag_error(err_flag, TK_DEVERR_TIMEOUT);
+                break;
+            }
+            const int64_t t = u / chunks;
+            const int ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
+            const int chn = min(kChunkCh, H - ch0);
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            if (!vec_ok[u]) continue;
-            uint4 o;
-            o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-            o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-            o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-            o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-            st_v4(out + t * row_bytes + static_cast<int64_t>(vbase + u * 32 + lane) * 16, o);
+            for (int q = 0; q < kVecs; ++q) {
+                const int vec = ct + q * 32 * kConsumerWarps;   // 8-channel vector within the unit
+                if (vec * 8 >= chn) break;
+                float acc[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+                const uint8_t* base = data + static_cast<size_t>(s) * stage_bytes + vec * 16;
+                for (int j = 0; j < k; ++j) {
+                    if (!meta[s].valid[j]) continue;
+                    const float wj = meta[s].w[j];
+                    const uint4 q4 = *reinterpret_cast<const uint4*>(base + j * kChunkBytes);
+                    acc[0] = __fmaf_rn(wj, lo_bf16(q4.x), acc[0]);
+                    acc[1] = __fmaf_rn(wj, hi_bf16(q4.x), acc[1]);
+                    acc[2] = __fmaf_rn(wj, lo_bf16(q4.y), acc[2]);
+                    acc[3] = __fmaf_rn(wj, hi_bf16(q4.y), acc[3]);
+                    acc[4] = __fmaf_rn(wj, lo_bf16(q4.z), acc[4]);
+                    acc[5] = __fmaf_rn(wj, hi_bf16(q4.z), acc[5]);
+                    acc[6] = __fmaf_rn(wj, lo_bf16(q4.w), acc[6]);
+                    acc[7] = __fmaf_rn(wj, hi_bf16(q4.w), acc[7]);
+                }
+                uint4 o;
+                o.x = pack_bf16x2(acc[0], acc[1]);
+                o.y = pack_bf16x2(acc[2], acc[3]);
+                o.z = pack_bf16x2(acc[4], acc[5]);
+                o.w = pack_bf16x2(acc[6], acc[7]);
+                st_v4(out + t * row_bytes + static_cast<int64_t>(ch0 + vec * 8) * 2, o);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
 }
 
-int reduce_grid(int64_t total_units) {
-    static int blocks_per_sm = 0;
-    if (blocks_per_sm == 0) {
-        int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, reduce_kernel, kRedThreads, 0) != cudaSuccess || b < 1) b = 1;
-        blocks_per_sm = b;
+struct LaunchShape {
+    int grid_cap = 0;   // SMs x resident CTAs for the current stage count
+    int S = 0;
+    int k = 0;
+};
+
+cudaError_t prepare(int k, LaunchShape& shape) {
+    static int configured_smem = 0;
+    const int S = stages_for(k);
+    const size_t smem = smem_bytes(k, S);
+    cudaError_t err = cudaSuccess;
+    if (static_cast<int>(smem) > configured_smem) {
+        err = cudaFuncSetAttribute(reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        configured_smem = static_cast<int>(smem);
     }
-    const int64_t want = (total_units + kRedWarps - 1) / kRedWarps;
-    const int64_t cap = static_cast<int64_t>(num_sms()) * blocks_per_sm;
-    return static_cast<int>(want < cap ? want : cap);
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel, kRedThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    shape.grid_cap = num_sms() * per_sm;
+    shape.S = S;
+    shape.k = k;
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -137,11 +240,18 @@ extern "C" tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slo
         return fail_arg("tk_reduce: y, slot_of and out must not be NULL");
     if (reinterpret_cast<uintptr_t>(y) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 16 != 0)
         return fail_arg("tk_reduce: y and out must be 16-byte aligned");
-    const int V = H / 8;
-    const int64_t units = static_cast<int64_t>(T) * ((V + 32 * kU - 1) / (32 * kU));
-    const int grid = reduce_grid(units);
-    cudaError_t err = launch_pdl(reduce_kernel, dim3(grid), dim3(kRedThreads), 0,
-                                 static_cast<cudaStream_t>(stream), static_cast<const uint8_t*>(y),
-                                 y_rows, slot_of, w, T, k, H, static_cast<uint8_t*>(out), err_flag);
+    static LaunchShape shapes[TK_MAX_TOPK + 1];
+    LaunchShape& shape = shapes[k];
+    if (shape.k != k) {
+        const cudaError_t e = prepare(k, shape);
+        if (e != cudaSuccess) return check_launch(e, "reduce_kernel setup");
+    }
+    const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
+    const int64_t units = static_cast<int64_t>(T) * chunks;
+    const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);
+    cudaError_t err = launch_pdl(reduce_kernel, dim3(grid), dim3(kRedThreads),
+                                 smem_bytes(k, shape.S), static_cast<cudaStream_t>(stream),
+                                 static_cast<const uint8_t*>(y), y_rows, slot_of, w, T, k, H,
+                                 shape.S, static_cast<uint8_t*>(out), err_flag);
     return check_launch(err, "reduce_kernel");
 }

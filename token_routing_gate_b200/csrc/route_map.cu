@@ -24,8 +24,10 @@ namespace {
 
 constexpr int kTileTokens = 256;               // tokens per tile
 constexpr int kTileWords = kTileTokens / 32;   // bitmap words per expert
-constexpr int kRouteThreads = 256;
+constexpr int kRouteThreads = 512;
+constexpr int kPairsPerThread = kTileTokens * TK_MAX_TOPK / kRouteThreads;  // 16
 constexpr int kScanThreads = 1024;
+constexpr int kScanBatch = 16;                 // column loads in flight per thread
 
 inline int num_tiles(int T) { return (T + kTileTokens - 1) / kTileTokens; }
 
@@ -36,34 +38,38 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     extern __shared__ int32_t cnt[];  // [E]
     pdl_wait();
     pdl_trigger();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-    // every row starts as "no token"; the scatter kernel fills the real rows afterwards
-    for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < rmax;
-         r += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        token_of[r] = -1;
-    __syncthreads();
     const int tile = blockIdx.x;
     const int64_t p0 = static_cast<int64_t>(tile) * kTileTokens * k;
     const int64_t p1 = min(static_cast<int64_t>(T), static_cast<int64_t>(tile + 1) * kTileTokens) * k;
-    // all 32 lanes of a warp run the same number of iterations, so __match_any_sync sees a full
-    // warp; lanes past the tile carry the sentinel -1
-    for (int64_t base = p0; base < p1; base += blockDim.x) {
-        const int64_t p = base + threadIdx.x;
-        int e = -1;
-        if (p < p1) {
-            e = topk_idx[p];
-            if (e < 0 || e >= E) {
-                flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
-                e = -1;
-            }
+    // all index loads of this thread first, so their latencies overlap
+    int e_reg[kPairsPerThread];
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        e_reg[i] = p < p1 ? topk_idx[p] : -1;
+    }
+    for (int e = threadIdx.x; e < E; e += kRouteThreads) cnt[e] = 0;
+    // every row starts as "no token"; the scatter kernel fills the real rows afterwards
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * kRouteThreads + threadIdx.x; r < rmax;
+         r += static_cast<int64_t>(gridDim.x) * kRouteThreads)
+        token_of[r] = -1;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        int e = e_reg[i];
+        if (p < p1 && (e < 0 || e >= E)) {
+            flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
+            e = -1;
         }
+        // the whole warp takes part (lanes past the tile carry -1)
         const unsigned peers = __match_any_sync(kFullMask, e);
-        const int lane = threadIdx.x & 31;
         if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt[e], __popc(peers));
     }
     __syncthreads();
     if (p0 < p1 || tile == 0) {
-        for (int e = threadIdx.x; e < E; e += blockDim.x)
+        for (int e = threadIdx.x; e < E; e += kRouteThreads)
             tile_counts[static_cast<int64_t>(tile) * E + e] = cnt[e];
     }
 }
@@ -86,22 +92,16 @@ route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align
         int32_t padded = 0;
         if (e < E) {
             int32_t run = 0;
-            int c = 0;
-            for (; c + 4 <= tiles; c += 4) {
-                const int32_t v0 = tile_counts[static_cast<int64_t>(c) * E + e];
-                const int32_t v1 = tile_counts[static_cast<int64_t>(c + 1) * E + e];
-                const int32_t v2 = tile_counts[static_cast<int64_t>(c + 2) * E + e];
-                const int32_t v3 = tile_counts[static_cast<int64_t>(c + 3) * E + e];
-                tile_counts[static_cast<int64_t>(c) * E + e] = run;
-                tile_counts[static_cast<int64_t>(c + 1) * E + e] = run + v0;
-                tile_counts[static_cast<int64_t>(c + 2) * E + e] = run + v0 + v1;
-                tile_counts[static_cast<int64_t>(c + 3) * E + e] = run + v0 + v1 + v2;
-                run += v0 + v1 + v2 + v3;
-            }
-            for (; c < tiles; ++c) {
-                const int32_t v = tile_counts[static_cast<int64_t>(c) * E + e];
-                tile_counts[static_cast<int64_t>(c) * E + e] = run;
-                run += v;
+            for (int c0 = 0; c0 < tiles; c0 += kScanBatch) {
+                int32_t v[kScanBatch];
+#pragma unroll
+                for (int i = 0; i < kScanBatch; ++i)
+                    v[i] = c0 + i < tiles ? tile_counts[static_cast<int64_t>(c0 + i) * E + e] : 0;
+#pragma unroll
+                for (int i = 0; i < kScanBatch; ++i) {
+                    if (c0 + i < tiles) tile_counts[static_cast<int64_t>(c0 + i) * E + e] = run;
+                    run += v[i];
+                }
             }
             counts[e] = run;
             padded = (run + align - 1) / align * align;
@@ -151,21 +151,32 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
     const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
-    for (int i = threadIdx.x; i < E * kTileWords; i += blockDim.x) bitmap[i] = 0u;
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
+    int e_reg[kPairsPerThread];
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        e_reg[i] = p < p1 ? topk_idx[p] : -1;
+    }
+    for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
+    for (int e = threadIdx.x; e < E; e += kRouteThreads)
         base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(tile) * E + e];
     __syncthreads();
-    for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
-        const int e = topk_idx[p];
-        if (e < 0 || e >= E) continue;  // flagged by the count kernel
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        const int e = e_reg[i];
+        if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged by the count kernel
         const int tl = static_cast<int>(p / k) - t0;
         const uint32_t bit = 1u << (tl & 31);
         const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
         if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
     }
     __syncthreads();
-    for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
-        const int e = topk_idx[p];
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        if (p >= p1) continue;
+        const int e = e_reg[i];
         if (e < 0 || e >= E) {
             slot_of[p] = -1;
             continue;

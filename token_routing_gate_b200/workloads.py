@@ -6,8 +6,10 @@ setting that the 機器之心 page ("剛剛，DeepSeek開始頻繁更新", secti
 expert-parallel benchmark (8K tokens, hidden 7168, top-8 of 256 experts, FP8 dispatch, BF16
 combine), plus a tiny case, a mid-size softmax case and a skewed-load case.
 
-All draws come from one torch.Generator seeded per workload (seed = 1000 + case number), on the
-CPU or on a CUDA device. The two devices give different (but each reproducible) streams.
+Token data (logits, x, y) is drawn from generators seeded with `seed` (1000 + case number);
+per-expert parameters (the selection bias, the skew ranking) from `param_seed`, so data-parallel
+shards that change `seed` still share one set of parameters. Draws run on the CPU or on a CUDA
+device; the two give different (but each reproducible) streams.
 """
 from dataclasses import dataclass, replace
 
@@ -26,7 +28,8 @@ class Workload:
     skew: bool          # add -2.2*ln(rank) over a random expert ranking to the logits
     align: int          # per-expert segment padding (rows)
     out_dtype: str      # expand output: "bf16" or "fp8"
-    seed: int
+    seed: int           # token data (logits, x, y); differs per data-parallel shard
+    param_seed: int = -1  # per-expert parameters (bias, skew ranking); -1 = same as seed
 
     @property
     def pairs(self) -> int:
@@ -66,12 +69,13 @@ def gate_inputs(wl: Workload, device="cpu"):
     2*ln(1/rank^1.1) = -2.2*ln(rank) for a random ranking 1..E of the experts."""
     g = _gen(wl.seed, device)
     logits = torch.randn(wl.T, wl.E, generator=g, device=device, dtype=torch.float32)
+    gp = _gen(wl.seed if wl.param_seed < 0 else wl.param_seed, "cpu")
     bias = None
     if wl.bias:
-        bias = torch.rand(wl.E, generator=g, device=device, dtype=torch.float32) * 0.2 - 0.1
+        bias = (torch.rand(wl.E, generator=gp, dtype=torch.float32) * 0.2 - 0.1).to(device)
     if wl.skew:
-        rank = torch.randperm(wl.E, generator=g, device=device).to(torch.float32) + 1.0
-        logits = logits + (-2.2 * torch.log(rank))[None, :]
+        rank = torch.randperm(wl.E, generator=gp).to(torch.float32) + 1.0
+        logits = logits + (-2.2 * torch.log(rank)).to(device)[None, :]
     return logits.contiguous(), bias
 
 
