@@ -115,6 +115,25 @@ TK_API tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int 
                        size_t workspace_bytes, int32_t* err_flag, void* stream);
 
 /*
+ * Allocation-free form of tk_route_map (the pages have no counterpart: this exists only for
+ * callers that cannot allocate device memory, such as a serving engine or plugin host that
+ * owns all device memory and hands a component only its inputs and outputs, or a
+ * latency-critical loop that must not call cudaMalloc, which can synchronise the device).
+ * Same arguments, results and errors as tk_route_map, without workspace: the scratch it needs
+ * is a 1 MiB array built into the library (every GPU that loads the library holds it until
+ * the process exits). It serves T and E with ceil(T/256) * E <= 262144 (e.g. T <= 262144 at
+ * E = 256, T <= 65536 at E = 1024); larger sizes return TK_ERR_INVALID_ARG and enqueue
+ * nothing. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it; make that first call before
+ * any stream capture. All calls on a device share the array and nothing in it needs to start
+ * at zero; calls that can overlap on the GPU (other streams, other host threads) race on it
+ * and must be serialised by the caller. The call allocates nothing.
+ */
+TK_API tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, int k, int align,
+                                     int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                                     int32_t* token_of, int32_t* err_flag, void* stream);
+
+/*
  * Fused expand / dispatch (147227.xyz "moe/": fused expand; 機器之心 "性能表現": FP8 dispatch
  * in the DeepSeek-V3 setting). Row t of x goes to rows slot_of[t*k+j], j < k, of out; padding
  * rows (token_of == -1 below offsets[E]) are written as zeros; rows at and beyond offsets[E]

@@ -253,3 +253,97 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
     }
     return TK_OK;
 }
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free variant of tk_route_map.
+//
+// Some callers cannot hand the library a workspace: a serving engine or plugin host that owns
+// every byte of device memory and passes a component only its input and output buffers, or a
+// latency-critical loop where a cudaMalloc (which can synchronise the device) is not allowed.
+// For them the tile-count matrix lives in a fixed array compiled into this library. Every GPU
+// that loads the library reserves it (1 MiB) until the process exits.
+//
+// The array's name is only a host-side stand-in in host code; its device address is looked up
+// with cudaGetSymbolAddress once per device (with that device current) on the first call on
+// that device, and cached. The kernels write every entry they later read, so nothing in the
+// array has to start at zero. All calls on one device share the array: calls that can overlap
+// on the GPU (other streams, other host threads) race on it and must be serialised by the
+// caller.
+// ------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+constexpr size_t kStaticScratchInts = 256 * 1024;  // 1 MiB of int32 tile counts
+static __device__ __align__(256) int32_t tk_route_static_scratch[kStaticScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of tk_route_static_scratch on the current device (looked up once per device).
+tk_status static_scratch(int32_t** out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return tk::check_launch(err, "tk_route_map_static: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return tk::fail_arg("tk_route_map_static: device index %d is beyond %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, tk_route_static_scratch);
+        if (err != cudaSuccess)
+            return tk::check_launch(err, "tk_route_map_static: cudaGetSymbolAddress");
+        g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = g_scratch_ptr[dev];
+    return TK_OK;
+}
+}  // namespace
+
+extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, int k, int align,
+                                         int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                                         int32_t* token_of, int32_t* err_flag, void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_route_map_static: T=%d must be >= 0", T);
+    if (E < 1 || E > TK_MAX_EXPERTS)
+        return fail_arg("tk_route_map_static: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (k < 1 || k > E || k > TK_MAX_TOPK)
+        return fail_arg("tk_route_map_static: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (align < 1 || align > 4096)
+        return fail_arg("tk_route_map_static: align=%d outside [1, 4096]", align);
+    const int64_t rmax = tk_max_rows(T, E, k, align);
+    if (rmax > INT32_MAX)
+        return fail_arg("tk_route_map_static: T*k + E*(align-1) = %lld exceeds int32", (long long)rmax);
+    const size_t need = route_map_workspace_bytes_impl(T, E) / sizeof(int32_t);
+    if (need > kStaticScratchInts)
+        return fail_arg("tk_route_map_static: T=%d, E=%d need %zu scratch entries but the built-in "
+                        "buffer holds %zu (at most %zu tiles of 256 tokens times E); use "
+                        "tk_route_map with a caller workspace", T, E, need, kStaticScratchInts,
+                        kStaticScratchInts / static_cast<size_t>(E));
+    if (counts == nullptr || offsets == nullptr)
+        return fail_arg("tk_route_map_static: counts and offsets must not be NULL");
+    if (T > 0 && (topk_idx == nullptr || slot_of == nullptr))
+        return fail_arg("tk_route_map_static: topk_idx and slot_of must not be NULL");
+    if (rmax > 0 && token_of == nullptr) return fail_arg("tk_route_map_static: token_of must not be NULL");
+    int32_t* tile_counts = nullptr;
+    const tk_status st = static_scratch(&tile_counts);
+    if (st != TK_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int tiles = num_tiles(T);
+    const int count_grid = tiles > 0 ? tiles : 1;
+    cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
+                                 static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
+                                 tile_counts, token_of, rmax, err_flag);
+    if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
+    err = launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tile_counts, tiles, E,
+                     align, counts, offsets);
+    if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
+    if (tiles > 0) {
+        const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
+        err = launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
+                         T, E, k, static_cast<const int32_t*>(tile_counts),
+                         static_cast<const int32_t*>(offsets), slot_of, token_of, err_flag);
+        if (err != cudaSuccess) return check_launch(err, "route_scatter_kernel");
+    }
+    return TK_OK;
+}

@@ -25,8 +25,8 @@ DEVERR_TIMEOUT = 16
 
 # every C entry point declared in include/tk_route.h
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
-               "tk_expand", "tk_reduce", "tk_status_str", "tk_last_error_detail",
-               "tk_abi_version")
+               "tk_route_map_static", "tk_expand", "tk_reduce", "tk_status_str",
+               "tk_last_error_detail", "tk_abi_version")
 
 
 class TkError(RuntimeError):
@@ -51,6 +51,8 @@ def _load():
     L.tk_route_map_workspace_bytes.restype = sz
     L.tk_route_map.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
     L.tk_route_map.restype = i32
+    L.tk_route_map_static.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.tk_route_map_static.restype = i32
     L.tk_expand.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
     L.tk_expand.restype = i32
     L.tk_reduce.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp, vp, vp]
