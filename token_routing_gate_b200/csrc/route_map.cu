@@ -3,8 +3,8 @@
 // mapping is one of the MoE routing ops).
 //
 // The pairs p = t*k + j are cut into tiles of kTileTokens tokens. Three short kernels:
-//   count   : one CTA per tile counts its pairs per expert in shared memory (warp-aggregated
-//             atomics; counts do not depend on their order) and writes a row of the
+//   count   : one CTA per tile counts its pairs per expert in shared memory (integer atomics,
+//             so the counts do not depend on their order) and writes a row of the
 //             [tiles x E] count matrix; the grid also fills token_of with -1.
 //   scan    : one CTA turns each column of the matrix into exclusive per-tile prefixes, sums
 //             the column into counts[e], rounds it up to the alignment and scans over experts
@@ -27,9 +27,15 @@ constexpr int kTileWords = kTileTokens / 32;   // bitmap words per expert
 constexpr int kRouteThreads = 512;
 constexpr int kPairsPerThread = kTileTokens * TK_MAX_TOPK / kRouteThreads;  // 16
 constexpr int kScanThreads = 1024;
-constexpr int kScanBatch = 16;                 // column loads in flight per thread
+constexpr int kScanBatch = 32;                 // column loads in flight per thread
 
 inline int num_tiles(int T) { return (T + kTileTokens - 1) / kTileTokens; }
+
+// The scan kernel gives each expert its own thread: E rounded up to whole warps.
+inline int scan_threads(int E) {
+    const int t = (E + 31) / 32 * 32;
+    return t < kScanThreads ? t : kScanThreads;
+}
 
 __global__ void __launch_bounds__(kRouteThreads)
 route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
@@ -42,11 +48,12 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     const int64_t p0 = static_cast<int64_t>(tile) * kTileTokens * k;
     const int64_t p1 = min(static_cast<int64_t>(T), static_cast<int64_t>(tile + 1) * kTileTokens) * k;
     // all index loads of this thread first, so their latencies overlap
+    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
     int e_reg[kPairsPerThread];
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
         const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        e_reg[i] = p < p1 ? topk_idx[p] : -1;
+        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
     }
     for (int e = threadIdx.x; e < E; e += kRouteThreads) cnt[e] = 0;
     // every row starts as "no token"; the scatter kernel fills the real rows afterwards
@@ -54,18 +61,17 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
          r += static_cast<int64_t>(gridDim.x) * kRouteThreads)
         token_of[r] = -1;
     __syncthreads();
-    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
         const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        int e = e_reg[i];
-        if (p < p1 && (e < 0 || e >= E)) {
+        if (p >= p1) continue;
+        const int e = e_reg[i];
+        if (e < 0 || e >= E) {
             flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
-            e = -1;
+            continue;
         }
-        // the whole warp takes part (lanes past the tile carry -1)
-        const unsigned peers = __match_any_sync(kFullMask, e);
-        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt[e], __popc(peers));
+        atomicAdd(&cnt[e], 1);  // integer counts: the order of the additions does not matter
     }
     __syncthreads();
     if (p0 < p1 || tile == 0) {
@@ -151,11 +157,12 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
     const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
+    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
     int e_reg[kPairsPerThread];
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
         const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        e_reg[i] = p < p1 ? topk_idx[p] : -1;
+        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
     }
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     for (int e = threadIdx.x; e < E; e += kRouteThreads)
@@ -163,6 +170,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
         const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
         const int e = e_reg[i];
         if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged by the count kernel
@@ -174,6 +182,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
         const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
         if (p >= p1) continue;
         const int e = e_reg[i];
@@ -241,7 +250,7 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
                                  tile_counts, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
-    err = launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tile_counts, tiles, E,
+    err = launch_pdl(route_scan_kernel, dim3(1), dim3(scan_threads(E)), 0, s, tile_counts, tiles, E,
                      align, counts, offsets);
     if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
     if (tiles > 0) {
