@@ -72,11 +72,12 @@ def _rand_inputs(wl, rng, rows=None):
     (1, 8, 1, 8, "softmax", False, 1, "bf16"),          # single token, k = 1, minimal H
     (3, 16, 16, 64, "softmax", False, 1, "bf16"),       # k = E
     (5, 32, 32, 128, "sigmoid", True, 1, "fp8"),        # k = E = warp width
+    (20000, 24, 3, 64, "sigmoid", True, 1, "bf16"),     # several tokens per gate warp
     (257, 37, 5, 264, "sigmoid", True, 1, "bf16"),      # ragged T, E % 32 != 0, H % 128 != 0
     (300, 1000, 12, 256, "softmax", False, 7, "bf16"),  # E close to the limit, odd alignment
     (64, 1024, 32, 128, "sigmoid", True, 128, "fp8"),   # largest E and k
     (513, 64, 6, 2048, "softmax", False, 128, "fp8"),   # many padding rows
-    (40, 48, 4, 20480, "sigmoid", False, 1, "bf16"),    # 40 KB rows: two bulk-copy stages
+    (40, 48, 4, 20480, "sigmoid", False, 16, "bf16"),   # 40 KB rows: two bulk-copy stages, padded
     (40, 48, 4, 9216, "sigmoid", True, 16, "fp8"),      # 9216 channels: two quantisation stages
 ])
 def test_shapes(T, E, k, H, score, bias, align, out):

@@ -91,98 +91,135 @@ __device__ __forceinline__ void sort_desc(uint64_t (&v)[EPL]) {
     }
 }
 
-// One warp per token. EPL = experts held per lane (E <= 32 * EPL).
+// One warp per token, tokens_per_warp consecutive tokens per warp (the grid is sized to one
+// wave of resident warps); the next token's logits are loaded while the current one is
+// processed. EPL = experts held per lane (E <= 32 * EPL).
 template <int EPL>
 __global__ void __launch_bounds__(kGateWarps * 32)
 gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
-                 int k, int score_fn, int renormalize, int32_t* __restrict__ topk_idx,
-                 float* __restrict__ topk_w) {
+                 int k, int score_fn, int renormalize, int tokens_per_warp,
+                 int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kGateWarps + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const float* row = logits + static_cast<int64_t>(t) * E;
+    const int64_t t_begin = (static_cast<int64_t>(blockIdx.x) * kGateWarps + (threadIdx.x >> 5)) * tokens_per_warp;
+    if (t_begin >= T) return;
+    const int64_t t_end = min(static_cast<int64_t>(T), t_begin + tokens_per_warp);
 
-    // Every real key maps above 0 (-inf maps to 0x007FFFFF), so 0 marks an absent expert
-    // (e >= E) or one already chosen, and real experts always win over absent ones.
-    uint64_t v[EPL];
+    float b[EPL];  // this lane's selection biases, shared by all tokens
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = i * 32 + lane;
-        v[i] = 0;
-        if (e < E) {
-            const float l = row[e];
-            const float key = bias != nullptr ? __fadd_rn(key_sigmoidf(l), bias[e]) : l;
-            v[i] = pack_key(ordered_key(key), e);
-        }
+        b[i] = (bias != nullptr && e < E) ? bias[e] : 0.0f;
     }
-    if (EPL > 1) sort_desc<EPL>(v);
-
-    int my_e = 0;  // lane j keeps the j-th winner
-    for (int j = 0; j < k; ++j) {
-        const uint32_t hi = static_cast<uint32_t>(v[0] >> 32);
-        const uint32_t m = __reduce_max_sync(kFullMask, hi);
-        const uint32_t lo = static_cast<uint32_t>(v[0]);
-        const uint32_t win = __reduce_max_sync(kFullMask, hi == m ? lo : 0u);  // ~e: lower e wins
-        if (lane == j) my_e = static_cast<int>(~win);
-        if (hi == m && lo == win) {  // the one lane holding the winner drops it
+    float lg[EPL];  // logits of the token being routed, then of the next one (prefetch)
 #pragma unroll
-            for (int i = 0; i + 1 < EPL; ++i) v[i] = v[i + 1];
-            v[EPL - 1] = 0;
-        }
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        lg[i] = e < E ? logits[t_begin * E + e] : 0.0f;
     }
-    const float my_l = lane < k ? row[my_e] : 0.0f;
 
-    // ---- weights (double), lanes 0..k-1 hold the chosen experts in order
-    const float top_l = __shfl_sync(kFullMask, my_l, 0);
-    double s = 0.0;
-    bool zero_all = false;
-    if (score_fn == TK_SCORE_SIGMOID) {
-        if (lane < k) s = 1.0 / (1.0 + exp(-static_cast<double>(my_l)));
-    } else {
-        // no bias with softmax, so the first winner holds the largest logit
-        if (top_l == -INFINITY || top_l != top_l) {
-            zero_all = true;
-        } else if (lane < k) {
-            s = exp(static_cast<double>(my_l) - static_cast<double>(top_l));
-        }
-    }
-    double denom;
-    if (renormalize) {
-        double v = s;
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        const float* row = logits + t * E;
+
+        // Every real key maps above 0 (-inf maps to 0x007FFFFF), so 0 marks an absent expert
+        // (e >= E) or one already chosen, and real experts always win over absent ones.
+        uint64_t v[EPL];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFullMask, v, off);
-        denom = v;
-    } else if (score_fn == TK_SCORE_SOFTMAX) {
-        // full softmax denominator over all E experts
-        double z = 0.0;
-        if (!zero_all) {
+        for (int i = 0; i < EPL; ++i) {
+            const int e = i * 32 + lane;
+            v[i] = 0;
+            if (e < E) {
+                const float l = lg[i];
+                const float key = bias != nullptr ? __fadd_rn(key_sigmoidf(l), b[i]) : l;
+                v[i] = pack_key(ordered_key(key), e);
+            }
+        }
+        if (t + 1 < t_end) {  // the registers are free again: start the next token's loads
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = i * 32 + lane;
-                if (e < E) z += exp(static_cast<double>(row[e]) - static_cast<double>(top_l));
+                lg[i] = e < E ? row[E + e] : 0.0f;
             }
         }
+        if (EPL > 1) sort_desc<EPL>(v);
+
+        int my_e = 0;  // lane j keeps the j-th winner
+        for (int j = 0; j < k; ++j) {
+            const uint32_t hi = static_cast<uint32_t>(v[0] >> 32);
+            const uint32_t m = __reduce_max_sync(kFullMask, hi);
+            const uint32_t lo = static_cast<uint32_t>(v[0]);
+            const uint32_t win = __reduce_max_sync(kFullMask, hi == m ? lo : 0u);  // ~e: lower e wins
+            if (lane == j) my_e = static_cast<int>(~win);
+            if (hi == m && lo == win) {  // the one lane holding the winner drops it
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFullMask, z, off);
-        denom = z;
-    } else {
-        denom = 1.0;
-    }
-    if (lane < k) {
-        const int64_t o = static_cast<int64_t>(t) * k + lane;
-        topk_idx[o] = my_e;
-        topk_w[o] = (zero_all || denom == 0.0) ? 0.0f : static_cast<float>(s / denom);
+                for (int i = 0; i + 1 < EPL; ++i) v[i] = v[i + 1];
+                v[EPL - 1] = 0;
+            }
+        }
+        const float my_l = lane < k ? row[my_e] : 0.0f;
+
+        // ---- weights (double), lanes 0..k-1 hold the chosen experts in order
+        const float top_l = __shfl_sync(kFullMask, my_l, 0);
+        double s = 0.0;
+        bool zero_all = false;
+        if (score_fn == TK_SCORE_SIGMOID) {
+            if (lane < k) s = 1.0 / (1.0 + exp(-static_cast<double>(my_l)));
+        } else {
+            // no bias with softmax, so the first winner holds the largest logit
+            if (top_l == -INFINITY || top_l != top_l) {
+                zero_all = true;
+            } else if (lane < k) {
+                s = exp(static_cast<double>(my_l) - static_cast<double>(top_l));
+            }
+        }
+        double denom;
+        if (renormalize) {
+            double acc = s;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFullMask, acc, off);
+            denom = acc;
+        } else if (score_fn == TK_SCORE_SOFTMAX) {
+            // full softmax denominator over all E experts
+            double z = 0.0;
+            if (!zero_all) {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) {
+                    const int e = i * 32 + lane;
+                    if (e < E) z += exp(static_cast<double>(row[e]) - static_cast<double>(top_l));
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(kFullMask, z, off);
+            denom = z;
+        } else {
+            denom = 1.0;
+        }
+        if (lane < k) {
+            const int64_t o = t * k + lane;
+            topk_idx[o] = my_e;
+            topk_w[o] = (zero_all || denom == 0.0) ? 0.0f : static_cast<float>(s / denom);
+        }
     }
 }
 
 template <int EPL>
 cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, int k, int score_fn,
                         int renormalize, int32_t* idx, float* w, cudaStream_t s) {
-    const dim3 grid((T + kGateWarps - 1) / kGateWarps);
+    // one wave: as many warps as fit on the GPU at once, each taking consecutive tokens
+    static int resident_warps = 0;
+    if (resident_warps == 0) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gate_topk_kernel<EPL>,
+                                                          kGateWarps * 32, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        resident_warps = per_sm * kGateWarps * num_sms();
+    }
+    const int tpw = (T + resident_warps - 1) / resident_warps;
+    const int warps = (T + tpw - 1) / tpw;
+    const dim3 grid((warps + kGateWarps - 1) / kGateWarps);
     return launch_pdl(gate_topk_kernel<EPL>, grid, dim3(kGateWarps * 32), 0, s, logits, bias, T, E,
-                      k, score_fn, renormalize, idx, w);
+                      k, score_fn, renormalize, tpw, idx, w);
 }
 
 }  // namespace
