@@ -2,7 +2,8 @@
 // slots (機器之心 "剛剛，DeepSeek開始頻繁更新", section "Tile Kernels": token-to-expert
 // mapping is one of the MoE routing ops).
 //
-// The pairs p = t*k + j are cut into tiles of kTileTokens tokens. Three short kernels:
+// The pairs p = t*k + j are cut into tiles of kTileTokens tokens. Three short kernels (the last
+// two run as one kernel, route_scan_scatter_kernel, while the batch has at most 128 tiles):
 //   count   : one CTA per tile counts its pairs per expert in shared memory (integer atomics,
 //             so the counts do not depend on their order) and writes a row of the
 //             [tiles x E] count matrix; the grid also fills token_of with -1.
@@ -28,6 +29,7 @@ constexpr int kRouteThreads = 512;
 constexpr int kPairsPerThread = kTileTokens * TK_MAX_TOPK / kRouteThreads;  // 16
 constexpr int kScanThreads = 1024;
 constexpr int kScanBatch = 32;                 // column loads in flight per thread
+constexpr int kFusedMaxTiles = 128;            // up to here every scatter CTA scans for itself
 
 inline int num_tiles(int T) { return (T + kTileTokens - 1) / kTileTokens; }
 
@@ -201,6 +203,126 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     }
 }
 
+// Scan and scatter in one kernel, for batches of at most kFusedMaxTiles tiles: every CTA reads
+// the whole (small) count matrix itself -- its own tile's prefix per expert, and every column's
+// total for the offsets -- instead of waiting for a separate scan kernel. CTA 0 also writes
+// counts[] and offsets[]. The slot arithmetic is the same as route_scan + route_scatter.
+__global__ void __launch_bounds__(kRouteThreads)
+route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int align,
+                          const int32_t* __restrict__ tile_counts, int tiles,
+                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                          int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
+                          int32_t* err_flag) {
+    extern __shared__ uint32_t smem[];
+    uint32_t* bitmap = smem;                                            // [E][kTileWords]
+    int32_t* base = reinterpret_cast<int32_t*>(smem + E * kTileWords);  // [E]
+    __shared__ int32_t warp_tot[kRouteThreads / 32];
+    __shared__ int32_t carry;
+    pdl_wait();
+    pdl_trigger();
+    const int tile = blockIdx.x;
+    const int t0 = tile * kTileTokens;
+    const int64_t p0 = static_cast<int64_t>(t0) * k;
+    const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
+    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
+    int e_reg[kPairsPerThread];
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
+    }
+    for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+
+    // ---- per expert: prefix over the tiles before this one, and the column total
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    for (int e0 = 0; e0 < E; e0 += kRouteThreads) {
+        const int e = e0 + threadIdx.x;
+        int32_t before = 0, total = 0;
+        if (e < E) {
+            for (int c0 = 0; c0 < tiles; c0 += kScanBatch) {
+                int32_t v[kScanBatch];
+#pragma unroll
+                for (int i = 0; i < kScanBatch; ++i)
+                    v[i] = c0 + i < tiles ? tile_counts[static_cast<int64_t>(c0 + i) * E + e] : 0;
+#pragma unroll
+                for (int i = 0; i < kScanBatch; ++i) {
+                    if (c0 + i < tile) before += v[i];
+                    total += v[i];
+                }
+            }
+        }
+        const int32_t padded = e < E ? (total + align - 1) / align * align : 0;
+        int32_t incl = padded;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t u = __shfl_up_sync(kFullMask, incl, off);
+            if (lane >= off) incl += u;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            constexpr int nw = kRouteThreads / 32;
+            int32_t u = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int32_t q = __shfl_up_sync(kFullMask, u, off);
+                if (lane >= off) u += q;
+            }
+            if (lane < nw) warp_tot[lane] = u;
+        }
+        __syncthreads();
+        const int32_t excl = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + incl - padded;
+        if (e < E) {
+            base[e] = excl + before;
+            if (tile == 0) {
+                counts[e] = total;
+                offsets[e] = excl;
+            }
+        }
+        const int32_t chunk_total = warp_tot[kRouteThreads / 32 - 1];
+        __syncthreads();
+        if (threadIdx.x == 0) carry += chunk_total;
+        __syncthreads();
+    }
+    if (tile == 0 && threadIdx.x == 0) offsets[E] = carry;
+
+    // ---- ranks inside the tile, as in route_scatter_kernel
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        const int e = e_reg[i];
+        if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged by the count kernel
+        const int tl = static_cast<int>(p / k) - t0;
+        const uint32_t bit = 1u << (tl & 31);
+        const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
+        if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        if (p >= p1) continue;
+        const int e = e_reg[i];
+        if (e < 0 || e >= E) {
+            slot_of[p] = -1;
+            continue;
+        }
+        const int t = static_cast<int>(p / k);
+        const int tl = t - t0;
+        const uint32_t* bm = bitmap + e * kTileWords;
+        int rank = __popc(bm[tl >> 5] & ((1u << (tl & 31)) - 1u));
+        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bm[w]);
+        const int32_t slot = base[e] + rank;
+        slot_of[p] = slot;
+        token_of[slot] = t;
+    }
+}
+
 }  // namespace
 
 size_t route_map_workspace_bytes_impl(int T, int E) {
@@ -250,6 +372,13 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
                                  tile_counts, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
+    if (tiles > 0 && tiles <= kFusedMaxTiles) {
+        const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
+        err = launch_pdl(route_scan_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s,
+                         topk_idx, T, E, k, align, static_cast<const int32_t*>(tile_counts), tiles,
+                         counts, offsets, slot_of, token_of, err_flag);
+        return check_launch(err, "route_scan_scatter_kernel");
+    }
     err = launch_pdl(route_scan_kernel, dim3(1), dim3(scan_threads(E)), 0, s, tile_counts, tiles, E,
                      align, counts, offsets);
     if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
