@@ -61,6 +61,12 @@ def _declare(L):
     L.tko_reduce_token.restype = i32
     L.tko_reduce.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp]
     L.tko_reduce.restype = i32
+    L.tko_balance_stats.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    L.tko_balance_stats.restype = i32
+    L.tko_tp_mask.argtypes = [vp, i32, i32, i32, i32, i32, vp]
+    L.tko_tp_mask.restype = i32
+    L.tko_reduce_backward.argtypes = [vp, vp, i64, vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    L.tko_reduce_backward.restype = i32
 
 
 def _c(a, dtype):
@@ -175,3 +181,43 @@ def reduce(y_bits, slot_of, w):
     if rc < 0:
         raise ValueError(f"tko_reduce rejected its arguments (rc={rc})")
     return out
+
+
+def balance_stats(logits, counts, k, score_fn):
+    """(P [E], f [E], loss) in float64."""
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    counts = _c(counts, np.int32)
+    P = np.empty(E, dtype=np.float64)
+    f = np.empty(E, dtype=np.float64)
+    loss = np.empty(1, dtype=np.float64)
+    if lib().tko_balance_stats(_p(logits), _p(counts), T, E, k, score_fn, _p(P), _p(f), _p(loss)) < 0:
+        raise ValueError("tko_balance_stats rejected its arguments")
+    return P, f, float(loss[0])
+
+
+def tp_mask(topk_idx, E, tp_size, tp_rank):
+    topk_idx = _c(topk_idx, np.int32)
+    T, k = topk_idx.shape
+    out = np.empty_like(topk_idx)
+    if lib().tko_tp_mask(_p(topk_idx), T, k, E, tp_size, tp_rank, _p(out)) < 0:
+        raise ValueError("tko_tp_mask rejected its arguments")
+    return out
+
+
+def reduce_backward(grad_bits, y_bits, slot_of, offsets, w, E):
+    """(d_y bits [y_rows, H] -- rows at and past offsets[E] left 0 --, d_w [T, k] fp32, rc)."""
+    grad_bits = _c(grad_bits, np.uint16)
+    y_bits = _c(y_bits, np.uint16)
+    slot_of = _c(slot_of, np.int32)
+    offsets = _c(offsets, np.int32)
+    w = _c(w, np.float32) if w is not None else None
+    T, H = grad_bits.shape
+    k = slot_of.shape[1]
+    d_y = np.zeros_like(y_bits)
+    d_w = np.empty((T, k), dtype=np.float32)
+    rc = lib().tko_reduce_backward(_p(grad_bits), _p(y_bits), y_bits.shape[0], _p(slot_of),
+                                   _p(offsets), _p(w), T, E, k, H, _p(d_y), _p(d_w))
+    if rc < 0:
+        raise ValueError("tko_reduce_backward rejected its arguments")
+    return d_y, d_w, rc

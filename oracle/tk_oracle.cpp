@@ -202,6 +202,7 @@ int64_t tko_max_rows(int T, int E, int k, int align) {
  * Pair p = t*k + j. One pass counts, a scan places each expert's segment (rounded up to a
  * multiple of align, padding rows keep token -1), a second pass in p order hands out slots, so
  * each segment lists its tokens in increasing order (a stable expert-major permutation).
+ * Expert -1 marks a masked pair (see tko_tp_mask): skipped without being an error.
  * ---------------------------------------------------------------------------------------- */
 int tko_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32_t* counts,
                   int32_t* offsets, int32_t* slot_of, int32_t* token_of) {
@@ -212,7 +213,10 @@ int tko_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32
     for (int e = 0; e < E; ++e) counts[e] = 0;
     for (int64_t p = 0; p < pairs; ++p) {
         const int e = topk_idx[p];
-        if (e < 0 || e >= E) { bad = 1; continue; }
+        if (e < 0 || e >= E) {
+            if (e != -1) bad = 1;  /* -1 = masked pair, not an error */
+            continue;
+        }
         counts[e] += 1;
     }
     offsets[0] = 0;
@@ -326,6 +330,98 @@ int tko_reduce(const uint16_t* y, int64_t y_rows, const int32_t* slot_of, const 
         const int64_t p = static_cast<int64_t>(t) * k;
         bad |= tko_reduce_token(y, y_rows, slot_of + p, w != nullptr ? w + p : nullptr, k, H,
                                 out + static_cast<int64_t>(t) * H);
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Load-balance statistics (147227.xyz "moe/": load-balance loss computation; the pages give no
+ * formula). The reading: the usual auxiliary balance loss of routed MoE layers -- the fraction
+ * of routed pairs per expert times the mean normalised routing score of that expert, summed
+ * and scaled so that perfectly balanced routing gives 1. Scores are the unbiased ones (the
+ * selection bias only steers selection).
+ * ---------------------------------------------------------------------------------------- */
+int tko_balance_stats(const float* logits, const int32_t* counts, int T, int E, int k,
+                      int score_fn, double* P, double* f, double* loss) {
+    if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+    if (score_fn != TKO_SCORE_SOFTMAX && score_fn != TKO_SCORE_SIGMOID) return -1;
+    std::vector<double> p(E);
+    for (int i = 0; i < E; ++i) P[i] = 0.0;
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + static_cast<int64_t>(t) * E;
+        double z = 0.0;
+        if (score_fn == TKO_SCORE_SOFTMAX) {
+            double m = -std::numeric_limits<double>::infinity();
+            for (int i = 0; i < E; ++i) m = std::max(m, static_cast<double>(l[i]));
+            for (int i = 0; i < E; ++i) { p[i] = std::exp(static_cast<double>(l[i]) - m); z += p[i]; }
+        } else {
+            for (int i = 0; i < E; ++i) { p[i] = 1.0 / (1.0 + std::exp(-static_cast<double>(l[i]))); z += p[i]; }
+        }
+        for (int i = 0; i < E; ++i) P[i] += p[i] / z;
+    }
+    double acc = 0.0;
+    for (int i = 0; i < E; ++i) {
+        P[i] = T > 0 ? P[i] / T : 0.0;
+        f[i] = T > 0 ? static_cast<double>(E) * counts[i] / (static_cast<double>(k) * T) : 0.0;
+        acc += f[i] * P[i];
+    }
+    *loss = acc;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Tensor-parallel mask (147227.xyz "moe/": tensor-parallel mask; no definition on the pages).
+ * The reading: experts are owned in E/tp_size contiguous groups; a rank keeps its own pairs,
+ * renumbered locally, and masks the rest with -1.
+ * ---------------------------------------------------------------------------------------- */
+int tko_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size, int tp_rank,
+                int32_t* out_idx) {
+    if (T < 0 || k < 1 || E < 1 || tp_size < 1 || E % tp_size != 0 || tp_rank < 0 ||
+        tp_rank >= tp_size)
+        return -1;
+    const int el = E / tp_size;
+    const int lo = tp_rank * el;
+    for (int64_t p = 0; p < static_cast<int64_t>(T) * k; ++p) {
+        const int e = topk_idx[p];
+        out_idx[p] = (e >= lo && e < lo + el) ? e - lo : -1;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Backward of the fused reduce (the training use of the fused expand/reduce; TileKernels is
+ * described as training and inference kernels, m.yhxrc.cn "簡介"). out = sum_j w_j y_j is
+ * linear in y and in w, so d_y_j = w_j * g and d_w_j = <g, y_j>. d_y is rounded like every bf16
+ * output here (fp32 product, then bf16); d_w is the dot product in double, rounded once.
+ * The backward of expand (a copy to k rows) is the unweighted reduce of the row gradients,
+ * which tko_reduce with w = NULL already states.
+ * ---------------------------------------------------------------------------------------- */
+int tko_reduce_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_rows,
+                        const int32_t* slot_of, const int32_t* offsets, const float* w, int T,
+                        int E, int k, int H, uint16_t* d_y, float* d_w) {
+    if (T < 0 || E < 1 || k < 1 || H <= 0 || y_rows < 0) return -1;
+    const int64_t rows = offsets[E];
+    std::memset(d_y, 0, static_cast<size_t>(rows) * H * sizeof(uint16_t));
+    int bad = 0;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t* g = grad_out + static_cast<int64_t>(t) * H;
+        for (int j = 0; j < k; ++j) {
+            const int64_t p = static_cast<int64_t>(t) * k + j;
+            const int64_t slot = slot_of[p];
+            if (slot < 0 || slot >= y_rows || slot >= rows) {
+                if (slot != -1) bad = 1;
+                d_w[p] = 0.0f;
+                continue;
+            }
+            const float wj = w != nullptr ? w[p] : 1.0f;
+            double dot = 0.0;
+            for (int c = 0; c < H; ++c) {
+                const float gc = bf16_to_float(g[c]);
+                dot += static_cast<double>(gc) * static_cast<double>(bf16_to_float(y[slot * H + c]));
+                d_y[slot * H + c] = tko_bf16_rne(wj * gc);
+            }
+            d_w[p] = static_cast<float>(dot);
+        }
     }
     return bad;
 }

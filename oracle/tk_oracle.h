@@ -10,7 +10,7 @@
  * Sources (web pages about DeepSeek's TileKernels; none prints code for these steps):
  *  - "刚刚！DeepSeek开源高性能GPU算子库TileKernels" (147227.xyz), section "1、moe/（14个算子）":
  *    the moe/ module covers top-k gating, expert scoring, token-to-expert mapping, fused
- *    expand/reduce (and a TP mask and a load-balance loss, not stated here).
+ *    expand/reduce, a tensor-parallel mask and a load-balance loss.
  *  - "剛剛，DeepSeek開始頻繁更新：Tile Kernels、DeepEP V2" (機器之心), section "Tile Kernels",
  *    feature list: gating = top-k expert selection and scoring; MoE routing = token-to-expert
  *    mapping, fused expansion/reduction and weight normalisation; section "性能表現": the
@@ -68,7 +68,8 @@ int64_t tko_max_rows(int T, int E, int k, int align);
 /* Token-to-expert map. counts[E]; offsets[E+1] = exclusive scan of counts rounded up to a
  * multiple of align; slot_of[T*k] = offsets[e] + (number of earlier pairs on expert e);
  * token_of[R_max] = token of each real row, -1 for padding rows and rows past offsets[E].
- * A pair whose expert lies outside [0,E) is not counted and gets slot -1 (returns 1). */
+ * A pair whose expert is -1 is masked: not counted, slot -1. Any other expert outside [0,E)
+ * is treated the same way and reported (returns 1). */
 int tko_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32_t* counts,
                   int32_t* offsets, int32_t* slot_of, int32_t* token_of);
 
@@ -91,6 +92,31 @@ int tko_reduce_token(const uint16_t* y, int64_t y_rows, const int32_t* slot_row,
 /* Reduce for all T tokens. */
 int tko_reduce(const uint16_t* y, int64_t y_rows, const int32_t* slot_of, const float* w, int T,
                int k, int H, uint16_t* out);
+
+/* ---- next rows: load-balance statistics, tensor-parallel mask, backward ---- */
+
+/* Load-balance statistics (147227.xyz "moe/" lists a load-balance loss among the routing ops;
+ * no formula on the pages). Per token the unbiased scores are normalised over all E experts:
+ * p[t,i] = softmax(l_t)_i, or sigmoid(l_ti) / sum_j sigmoid(l_tj) for sigmoid scoring. Then
+ *   P[i] = (1/T) sum_t p[t,i],  f[i] = E * counts[i] / (k*T),  loss = sum_i f[i] * P[i]
+ * (loss = 1 for perfectly balanced routing). All in double; T = 0 gives zeros. */
+int tko_balance_stats(const float* logits, const int32_t* counts, int T, int E, int k,
+                      int score_fn, double* P, double* f, double* loss);
+
+/* Tensor-parallel expert mask: experts are split into tp_size contiguous groups of E/tp_size;
+ * rank tp_rank keeps pairs on its own group, renumbered to local indices 0..E/tp_size-1, and
+ * marks every other pair -1 (a masked pair, which the route map skips). */
+int tko_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size, int tp_rank,
+                int32_t* out_idx);
+
+/* Backward of the weighted reduce out[t] = sum_j w[t,j] * y[slot_of[t,j]]:
+ *   d_y[slot_of[t,j], c] = bf16( fp32(w[t,j] * g[t,c]) )      (w = NULL: weight 1)
+ *   d_w[t,j] = fp32( sum_c double(g[t,c]) * double(y[slot_of[t,j], c]) )  (summed in c order)
+ * Rows of d_y in [0, offsets[E]) that no pair references (padding) are zero; rows at and
+ * beyond offsets[E] are not written. A pair with an out-of-range slot gets d_w = 0. */
+int tko_reduce_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_rows,
+                        const int32_t* slot_of, const int32_t* offsets, const float* w, int T,
+                        int E, int k, int H, uint16_t* d_y, float* d_w);
 
 #ifdef __cplusplus
 }

@@ -405,3 +405,131 @@ def test_fp8_expand_same_codes_in_every_slot(oracle_lib):
             np.testing.assert_array_equal(s[slot_of[t, j]], st)
     pad = np.where(token_of[:offsets[-1]] == -1)[0]
     assert np.all(q[pad] == 0) and np.all(s[pad] == 0)
+
+
+# ---------------------------------------------------------------- load-balance statistics
+def test_balance_stats_uniform_scores_closed_form(oracle_lib):
+    # equal logits: every normalised score is 1/E, so P = 1/E and loss = sum f / E = 1
+    T, E, k = 37, 12, 3
+    rng = np.random.default_rng(20)
+    counts = np.bincount(rng.integers(0, E, T * k), minlength=E).astype(np.int32)
+    for fn in (oracle_lib.SOFTMAX, oracle_lib.SIGMOID):
+        P, f, loss = oracle_lib.balance_stats(np.full((T, E), 0.3, np.float32), counts, k, fn)
+        np.testing.assert_allclose(P, 1.0 / E, rtol=1e-14)
+        np.testing.assert_allclose(f, E * counts / (k * T), rtol=1e-14)
+        assert abs(loss - 1.0) < 1e-12
+
+
+def test_balance_stats_against_library(oracle_lib):
+    rng = np.random.default_rng(21)
+    T, E, k = 200, 40, 6
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    idx, _ = oracle_lib.gate_topk(logits, None, k, oracle_lib.SOFTMAX)
+    counts, *_ = oracle_lib.route_map(idx, E, 1)
+    P, f, loss = oracle_lib.balance_stats(logits, counts, k, oracle_lib.SOFTMAX)
+    p = scipy.special.softmax(logits.astype(np.float64), axis=1)
+    np.testing.assert_allclose(P, p.mean(0), rtol=1e-12)
+    np.testing.assert_allclose(f, np.bincount(idx.ravel(), minlength=E) * E / (k * T), rtol=1e-14)
+    assert abs(loss - float(np.dot(f, P))) < 1e-12
+    s = scipy.special.expit(logits.astype(np.float64))
+    P2, _, _ = oracle_lib.balance_stats(logits, counts, k, oracle_lib.SIGMOID)
+    np.testing.assert_allclose(P2, (s / s.sum(1, keepdims=True)).mean(0), rtol=1e-12)
+    assert abs(P2.sum() - 1.0) < 1e-12
+
+
+def test_balance_stats_all_on_one_expert(oracle_lib):
+    # every token routes only to expert 0 with (almost) all of its score: loss -> E
+    T, E = 50, 8
+    logits = np.full((T, E), -60.0, np.float32)
+    logits[:, 0] = 60.0
+    counts = np.zeros(E, np.int32)
+    counts[0] = T
+    P, f, loss = oracle_lib.balance_stats(logits, counts, 1, oracle_lib.SOFTMAX)
+    assert f[0] == E and abs(P[0] - 1.0) < 1e-12 and abs(loss - E) < 1e-9
+
+
+# ---------------------------------------------------------------- tensor-parallel mask
+def test_tp_mask_partitions_every_pair(oracle_lib):
+    rng = np.random.default_rng(22)
+    T, E, k, tp = 90, 24, 4, 3
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    owners = np.zeros_like(idx)
+    rebuilt = np.full_like(idx, -100)
+    for r in range(tp):
+        m = oracle_lib.tp_mask(idx, E, tp, r)
+        kept = m >= 0
+        assert np.all(m[kept] < E // tp)
+        owners += kept
+        rebuilt[kept] = m[kept] + r * (E // tp)
+    assert np.all(owners == 1)            # each pair kept by exactly one rank
+    np.testing.assert_array_equal(rebuilt, idx)
+    with pytest.raises(ValueError):
+        oracle_lib.tp_mask(idx, E, 5, 0)  # E not divisible
+
+
+def test_masked_pairs_are_skipped_by_the_route_map(oracle_lib):
+    idx = np.array([[0, -1], [-1, 2], [1, 0]], dtype=np.int32)
+    counts, offsets, slot_of, token_of, rc = oracle_lib.route_map(idx, 3, 1)
+    assert rc == 0                        # -1 is a masked pair, not an error
+    assert counts.tolist() == [2, 1, 1] and offsets.tolist() == [0, 2, 3, 4]
+    assert slot_of.tolist() == [[0, -1], [-1, 3], [2, 1]]
+
+
+# ---------------------------------------------------------------- reduce backward
+def _route(oracle_lib, T, E, k, align, seed):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, offsets, slot_of, token_of, _ = oracle_lib.route_map(idx, E, align)
+    return idx, offsets, slot_of, token_of
+
+
+def test_reduce_backward_adjoint_identity(oracle_lib):
+    # <g, reduce(y; w)> = sum_tj w_tj * d_w_tj exactly in real arithmetic (reduce is linear in y)
+    T, E, k, H = 60, 10, 3, 64
+    rng = np.random.default_rng(23)
+    _, offsets, slot_of, token_of = _route(oracle_lib, T, E, k, 1, 23)
+    R = int(offsets[-1])
+    y = _bf16_bits(rng.standard_normal((R, H)))
+    g = _bf16_bits(rng.standard_normal((T, H)))
+    w = rng.uniform(0, 1, (T, k)).astype(np.float32)
+    d_y, d_w, rc = oracle_lib.reduce_backward(g, y, slot_of, offsets, w, E)
+    assert rc == 0
+    yf = _bits_to_f32(y).astype(np.float64)
+    gf = _bits_to_f32(g).astype(np.float64)
+    exact_dw = np.einsum("tc,tjc->tj", gf, yf[slot_of])
+    np.testing.assert_allclose(d_w, exact_dw.astype(np.float32), rtol=0, atol=0)
+    lhs = float(np.sum(gf * np.einsum("tj,tjc->tc", w.astype(np.float64), yf[slot_of])))
+    rhs = float(np.sum(w.astype(np.float64) * exact_dw))
+    assert abs(lhs - rhs) <= 1e-9 * max(1.0, abs(lhs))
+    # d_y rows: w * g rounded to bf16, one row per pair
+    for t in range(T):
+        for j in range(k):
+            want = oracle_lib.bf16_rne((w[t, j] * _bits_to_f32(g[t])).astype(np.float32))
+            np.testing.assert_array_equal(d_y[slot_of[t, j]], want)
+
+
+def test_reduce_backward_unit_weights_and_padding(oracle_lib):
+    T, E, k, H, align = 33, 6, 2, 16, 8
+    rng = np.random.default_rng(24)
+    _, offsets, slot_of, token_of = _route(oracle_lib, T, E, k, align, 24)
+    R = int(offsets[-1])
+    y = _bf16_bits(rng.standard_normal((tko_rows := T * k + E * (align - 1), H)))
+    g = _bf16_bits(rng.standard_normal((T, H)))
+    d_y, d_w, rc = oracle_lib.reduce_backward(g, y, slot_of, offsets, None, E)
+    for t in range(T):
+        for j in range(k):
+            np.testing.assert_array_equal(d_y[slot_of[t, j]], g[t])    # weight 1: a copy
+    pad = np.where(token_of[:R] == -1)[0]
+    assert len(pad) > 0 and np.all(d_y[pad] == 0)
+    # the backward of expand is the unweighted reduce: <expand(x), G> = <x, reduce(G)> exactly
+    x = _bf16_bits(rng.standard_normal((T, H)))
+    xe, _ = oracle_lib.expand(x, slot_of, offsets, E, align)
+    G = _bf16_bits(rng.standard_normal((tko_rows, H)))
+    back = oracle_lib.reduce(G, slot_of, None)
+    Gf = _bits_to_f32(G).astype(np.float64)
+    lhs = float(np.sum(_bits_to_f32(xe).astype(np.float64) * Gf))
+    rhs_exact = float(np.sum(_bits_to_f32(x).astype(np.float64) * Gf[slot_of].sum(1)))
+    assert abs(lhs - rhs_exact) <= 1e-9 * max(1.0, abs(lhs))
+    # and the fp32/bf16 reduce of G is that sum rounded (within the reduce's own bound)
+    exact = Gf[slot_of].sum(1)
+    assert np.all(np.abs(_bits_to_f32(back) - exact) <= k * 2.0 ** -24 * np.abs(Gf[slot_of]).sum(1) + np.abs(exact) * 2.0 ** -8)
