@@ -54,7 +54,7 @@ typedef enum tk_score_fn { TK_SCORE_SOFTMAX = 0, TK_SCORE_SIGMOID = 1 } tk_score
 typedef enum tk_out_dtype { TK_OUT_BF16 = 0, TK_OUT_FP8_E4M3 = 1 } tk_out_dtype;
 
 /* Bits ORed into *err_flag by the kernels. */
-#define TK_DEVERR_EXPERT_RANGE 1 /* tk_route_map: a topk_idx entry outside [0,E) (pair skipped, slot -1) */
+#define TK_DEVERR_EXPERT_RANGE 1 /* tk_route_map: a topk_idx entry outside [0,E), other than -1 (skipped, slot -1) */
 #define TK_DEVERR_DUP_EXPERT 2   /* tk_route_map: a token lists one expert twice (slots then overlap) */
 #define TK_DEVERR_SLOT_RANGE 4   /* tk_expand / tk_reduce: a slot outside the buffer (skipped) */
 #define TK_DEVERR_ROWS_RANGE 8   /* tk_expand: offsets[E] above the worst-case row count (clamped) */
@@ -103,7 +103,8 @@ TK_API size_t tk_route_map_workspace_bytes(int T, int E, int k);
  *             ceil(counts[e]/align)*align; offsets[E] = R, the rows in use
  *   slot_of   device, int32 [T*k]: row of pair p = offsets[e] + (number of pairs p' < p on
  *             expert e), so each segment lists its tokens in increasing order (-1 for a pair
- *             whose expert is out of range)
+ *             whose expert is out of range). Expert -1 marks a masked pair (tk_tp_mask): it is
+ *             skipped like an out-of-range one but sets no error bit.
  *   token_of  device, int32 [tk_max_rows()]: token of each row, -1 for padding rows and for
  *             rows at and beyond R
  *   workspace device, at least tk_route_map_workspace_bytes(T, E, k) bytes, 16-byte
@@ -168,6 +169,61 @@ TK_API tk_status tk_expand(const void* x, const int32_t* slot_of, const int32_t*
  */
 TK_API tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slot_of, const float* w, int T,
                     int k, int H, void* out, int32_t* err_flag, void* stream);
+
+/*
+ * Load-balance statistics (147227.xyz "moe/": load-balance loss computation; no formula on the
+ * pages -- this is the usual auxiliary balance loss of routed MoE layers). With p[t,i] the
+ * unbiased scores of token t normalised over all E experts (softmax, or sigmoid divided by its
+ * row sum):
+ *   P[i] = (1/T) sum_t p[t,i],   f[i] = E * counts[i] / (k*T),   loss = sum_i f[i] * P[i]
+ * so perfectly balanced routing gives loss = 1. Computed in double (deterministic: fixed
+ * 64-token tiles and fixed-order sums), written as fp32.
+ *   logits    device, fp32 [T, E] (the gate's logits; the selection bias is not used)
+ *   counts    device, int32 [E] (tk_route_map's counts)
+ *   P, f      device, fp32 [E];  loss  device, fp32 [1]
+ *   workspace device, tk_balance_stats_workspace_bytes(T, E) bytes, 16-byte aligned
+ */
+TK_API size_t tk_balance_stats_workspace_bytes(int T, int E);
+TK_API tk_status tk_balance_stats(const float* logits, const int32_t* counts, int T, int E, int k,
+                                  int score_fn, float* P, float* f, float* loss, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
+ * Tensor-parallel expert mask (147227.xyz "moe/": tensor-parallel mask; no definition on the
+ * pages). Experts are owned in tp_size contiguous groups of E/tp_size; for rank tp_rank,
+ * out_idx = topk_idx - tp_rank*E/tp_size where the expert is in the rank's group, else -1 (a
+ * masked pair, which tk_route_map skips). Route the result with E/tp_size experts.
+ * out_idx may equal topk_idx (in place). tp_size must divide E.
+ */
+TK_API tk_status tk_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size,
+                            int tp_rank, int32_t* out_idx, void* stream);
+
+/*
+ * Backward of tk_reduce (its inputs y and w), for training: with g = d(loss)/d(out) [T, H],
+ *   d_y[slot_of[t,j], c] = bf16(fp32(w[t,j] * g[t,c]))       (w = NULL: weight 1)
+ *   d_w[t,j]             = fp32(sum_c g[t,c] * y[slot_of[t,j], c])   (double accumulation)
+ *   grad_out  device, bf16 [T, H];  y  device, bf16 [y_rows, H];  d_y  device, bf16 [y_rows, H]
+ *   offsets, token_of  from tk_route_map, or both NULL: with them, padding rows of d_y below
+ *             offsets[E] are zeroed, so d_y is complete up to offsets[E]; rows no pair
+ *             references are otherwise not written
+ *   d_w       device, fp32 [T, k] (0 for a pair whose slot is -1 or out of range)
+ *   workspace device, tk_reduce_backward_workspace_bytes(T, k) bytes, 16-byte aligned
+ * d_w is deterministic; it matches the exact dot product rounded to fp32 within 1 ulp.
+ */
+TK_API size_t tk_reduce_backward_workspace_bytes(int T, int k);
+TK_API tk_status tk_reduce_backward(const void* grad_out, const void* y, int64_t y_rows,
+                                    const int32_t* slot_of, const int32_t* offsets,
+                                    const int32_t* token_of, const float* w, int T, int E, int k,
+                                    int H, void* d_y, float* d_w, void* workspace,
+                                    size_t workspace_bytes, int32_t* err_flag, void* stream);
+
+/*
+ * Backward of tk_expand (bf16): d_x[t] = sum_j d_xe[slot_of[t,j]], the unweighted reduce of the
+ * gradient rows -- same kernel and arithmetic as tk_reduce with w = NULL.
+ */
+TK_API tk_status tk_expand_backward(const void* d_xe, int64_t xe_rows, const int32_t* slot_of,
+                                    int T, int k, int H, void* d_x, int32_t* err_flag,
+                                    void* stream);
 
 /* Name of a status code (static string). */
 TK_API const char* tk_status_str(int status);

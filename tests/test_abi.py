@@ -136,3 +136,30 @@ def test_binding_raises_with_detail(tk):
     with pytest.raises(tk.TkError) as ei:
         tk._check("tk_reduce", tk.lib.tk_reduce(FAKE, 1, FAKE, None, 4, 0, 256, FAKE, None, None))
     assert "k=0" in str(ei.value)
+
+
+def test_next_rows_reject_bad_arguments(tk):
+    L = tk.lib
+    ws = L.tk_balance_stats_workspace_bytes(128, 16)
+    assert ws == 2 * 16 * 8
+    ok = [FAKE, FAKE, 128, 16, 2, 1, FAKE, FAKE, FAKE, FAKE, ws, None]
+    for i, v, what in [(4, 17, "k"), (5, 3, "score_fn"), (10, ws - 8, "workspace"), (9, MISALIGNED, "aligned"),
+                       (1, None, "NULL")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_balance_stats(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode()
+    for args, what in [((FAKE, 10, 2, 16, 3, 0, FAKE, None), "divide"),
+                       ((FAKE, 10, 2, 16, 4, 4, FAKE, None), "tp_rank"),
+                       ((FAKE, 10, 0, 16, 4, 0, FAKE, None), "k")]:
+        assert L.tk_tp_mask(*args) == 1 and what in L.tk_last_error_detail().decode()
+    wsb = L.tk_reduce_backward_workspace_bytes(64, 4)
+    assert wsb == 64 * 4 * 4 * 8
+    ok = [FAKE, FAKE, 256, FAKE, FAKE, FAKE, None, 64, 16, 4, 256, FAKE, FAKE, FAKE, wsb, None, None]
+    for i, v, what in [(10, 12, "H"), (9, 0, "k"), (14, wsb - 8, "workspace"), (0, MISALIGNED, "aligned"),
+                       (4, None, "together"), (13, None, "NULL")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_reduce_backward(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode()
+    assert L.tk_expand_backward(FAKE, 10, FAKE, 4, 0, 256, FAKE, None, None) == 1

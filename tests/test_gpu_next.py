@@ -1,0 +1,130 @@
+"""Parity of the next routing ops with the oracle: load-balance statistics, the tensor-parallel
+expert mask (and routing of its masked output), and the backward of reduce and expand."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import bf16_bits, bf16_ulp_diff, bits_to_f32
+from token_routing_gate_b200 import tk
+from token_routing_gate_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+ULP32 = 2.0 ** -23  # both sides accumulate in double; the fp32 outputs differ by rounding only
+
+
+@pytest.mark.parametrize("wl", [W.V3, W.MID, W.TINY.with_(T=77, E=37, k=5),
+                                W.SKEW.with_(T=1000)], ids=lambda w: w.name)
+def test_balance_stats(wl):
+    logits, bias = W.gate_inputs(wl, "cuda")
+    idx, _ = tk.gate_topk(logits, wl.k, wl.score, bias)
+    rm = tk.route_map(idx, wl.E, 1)
+    P, f, loss = tk.balance_stats(logits, rm.counts, wl.k, wl.score)
+    P2, f2, loss2 = tk.balance_stats(logits, rm.counts, wl.k, wl.score)
+    torch.cuda.synchronize()
+    assert torch.equal(P, P2) and torch.equal(loss, loss2)          # deterministic
+    fn = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
+    Pr, fr, lr = oracle.balance_stats(logits.cpu().numpy(), rm.counts.cpu().numpy(), wl.k, fn)
+    np.testing.assert_allclose(P.cpu().numpy(), Pr, rtol=ULP32, atol=0)
+    np.testing.assert_allclose(f.cpu().numpy(), fr, rtol=ULP32, atol=0)
+    assert abs(loss.item() - lr) <= ULP32 * abs(lr)
+
+
+def test_balance_stats_empty_batch():
+    counts = torch.zeros(16, dtype=torch.int32, device="cuda")
+    P, f, loss = tk.balance_stats(torch.empty(0, 16, device="cuda"), counts, 2, "softmax")
+    torch.cuda.synchronize()
+    assert (P == 0).all() and (f == 0).all() and loss.item() == 0.0
+
+
+@pytest.mark.parametrize("tp", [1, 2, 8])
+def test_tp_mask_then_route(tp):
+    wl = W.V3.with_(T=3000)
+    logits, bias = W.gate_inputs(wl, "cuda")
+    idx, _ = tk.gate_topk(logits, wl.k, wl.score, bias)
+    idx_h = idx.cpu().numpy()
+    owned = torch.zeros_like(idx)
+    for r in range(tp):
+        m = tk.tp_mask(idx, wl.E, tp, r)
+        ref = oracle.tp_mask(idx_h, wl.E, tp, r)
+        np.testing.assert_array_equal(m.cpu().numpy(), ref)
+        owned += (m >= 0).int()
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        rm = tk.route_map(m, wl.E // tp, 128, err_flag=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0                                      # masked pairs are not errors
+        counts, offsets, slot_of, token_of, rc = oracle.route_map(ref, wl.E // tp, 128)
+        assert rc == 0
+        np.testing.assert_array_equal(rm.counts.cpu().numpy(), counts)
+        np.testing.assert_array_equal(rm.offsets.cpu().numpy(), offsets)
+        np.testing.assert_array_equal(rm.slot_of.cpu().numpy(), slot_of)
+        np.testing.assert_array_equal(rm.token_of.cpu().numpy(), token_of)
+    assert (owned == 1).all()
+    inplace = idx.clone()
+    tk.tp_mask(inplace, wl.E, tp, tp - 1, out=inplace)
+    np.testing.assert_array_equal(inplace.cpu().numpy(), oracle.tp_mask(idx_h, wl.E, tp, tp - 1))
+
+
+@pytest.mark.parametrize("T,E,k,H,align,weighted", [
+    (300, 16, 4, 264, 8, True),      # ragged chunk, padding rows
+    (2048, 256, 8, 7168, 1, True),   # DeepSeek-V3 row shape
+    (129, 8, 1, 2048, 4, False),     # k = 1, unit weights
+    (40, 64, 32, 1024, 1, True),     # largest k: one stage per CTA
+])
+def test_reduce_backward(T, E, k, H, align, weighted):
+    wl = W.V3.with_(T=T, E=E, k=k, H=H, align=align, bias=False, seed=T + H)
+    logits, _ = W.gate_inputs(wl, "cuda")
+    idx, w = tk.gate_topk(logits, k, "sigmoid")
+    rm = tk.route_map(idx, E, align)
+    rows = wl.max_rows
+    y = W.expert_outputs(wl, "cuda", rows=rows)
+    g = W.activations(wl.with_(seed=wl.seed + 5), "cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    d_y = torch.full_like(y, 7.0)                                      # garbage where not written
+    d_y, d_w = tk.reduce_backward(g, y, rm.slot_of, w if weighted else None, E, rm=rm, d_y=d_y,
+                                  err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    offsets = rm.offsets.cpu().numpy()
+    R = int(offsets[-1])
+    dy_ref, dw_ref, rc = oracle.reduce_backward(bf16_bits(g), bf16_bits(y), rm.slot_of.cpu().numpy(),
+                                                offsets, w.cpu().numpy() if weighted else None, E)
+    assert rc == 0
+    np.testing.assert_array_equal(bf16_bits(d_y)[:R], dy_ref[:R])
+    np.testing.assert_allclose(d_w.cpu().numpy(), dw_ref, rtol=ULP32, atol=0)
+    d_w2 = tk.reduce_backward(g, y, rm.slot_of, w if weighted else None, E, rm=rm)[1]
+    torch.cuda.synchronize()
+    assert torch.equal(d_w, d_w2)                                      # deterministic
+
+
+def test_reduce_backward_full_size_properties():
+    wl = W.V3
+    logits, bias = W.gate_inputs(wl, "cuda")
+    idx, w = tk.gate_topk(logits, wl.k, wl.score, bias)
+    rm = tk.route_map(idx, wl.E, 1)
+    y = W.expert_outputs(wl, "cuda")
+    g = W.activations(wl.with_(seed=77), "cuda")
+    d_y, d_w = tk.reduce_backward(g, y, rm.slot_of, w, wl.E, rm=rm)
+    torch.cuda.synchronize()
+    sl = rm.slot_of.long()
+    # d_y[slot] = bf16(w * g) for every pair (fp32 product, round to nearest even)
+    want = (w[:, :, None] * g.float()[:, None, :]).to(torch.bfloat16)
+    assert torch.equal(d_y[sl].view(torch.int16), want.view(torch.int16))
+    # d_w = <g, y[slot]>: exact products summed in double, then fp32
+    exact = torch.einsum("tc,tjc->tj", g.double(), y[sl].double())
+    assert torch.all((d_w.double() - exact).abs() <= ULP32 * exact.abs() + 1e-30)
+
+
+def test_expand_backward_is_the_unweighted_reduce():
+    wl = W.V3.with_(T=1024, align=128, skew=True)
+    logits, _ = W.gate_inputs(wl, "cuda")
+    idx, _ = tk.gate_topk(logits, wl.k, "sigmoid")
+    rm = tk.route_map(idx, wl.E, wl.align)
+    d_xe = W.expert_outputs(wl, "cuda")
+    d_x = tk.expand_backward(d_xe, rm.slot_of)
+    ref_gpu = tk.reduce(d_xe, rm.slot_of, None)
+    torch.cuda.synchronize()
+    assert torch.equal(d_x.view(torch.int16), ref_gpu.view(torch.int16))
+    ref = oracle.reduce(bf16_bits(d_xe), rm.slot_of.cpu().numpy(), None)
+    np.testing.assert_array_equal(bf16_bits(d_x), ref)

@@ -1,0 +1,224 @@
+// Load-balance statistics and the tensor-parallel expert mask, the two small routing ops that
+// the TileKernels moe/ module lists next to gating and expand/reduce (147227.xyz "刚刚！DeepSeek
+// 开源高性能GPU算子库TileKernels", section "moe/": tensor-parallel mask, load-balance loss
+// computation). The pages give no formulas; the readings are stated at the C declarations.
+//
+// Balance statistics, deterministic and in double:
+//   balance_partial_kernel: one CTA per tile of 64 tokens, one warp per 8 tokens. Each lane
+//     holds experts lane, lane+32, ... of a token, normalises their unbiased scores over the
+//     row (warp reductions) and adds them into per-lane double accumulators; the CTA then sums
+//     its 8 warps in order and writes one row of a [tiles x E] partial-sum matrix.
+//   balance_final_kernel: one CTA sums each column in tile order, forms P, f and the loss with
+//     a fixed-order tree. The tiling depends on T only, so results do not depend on the GPU.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "tk_device.cuh"
+
+namespace tk {
+namespace {
+
+constexpr int kStatTileTokens = 64;
+constexpr int kStatWarps = 8;
+constexpr int kStatTokensPerWarp = kStatTileTokens / kStatWarps;
+constexpr int kFinalThreads = 1024;
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFullMask, v, off);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFullMask, v, off));
+    return v;
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(kStatWarps * 32)
+balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score_fn,
+                       double* __restrict__ partial) {
+    extern __shared__ double wsum[];  // [kStatWarps][E]
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    double acc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.0;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kStatTileTokens + warp * kStatTokensPerWarp;
+    for (int q = 0; q < kStatTokensPerWarp; ++q) {
+        const int64_t t = t0 + q;
+        if (t >= T) break;
+        const float* row = logits + t * E;
+        float l[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = i * 32 + lane;
+            l[i] = e < E ? row[e] : -INFINITY;
+        }
+        double s[EPL];
+        double z = 0.0;
+        if (score_fn == TK_SCORE_SOFTMAX) {
+            float m = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) m = fmaxf(m, l[i]);
+            m = warp_max_f(m);
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = i * 32 + lane;
+                s[i] = e < E ? exp(static_cast<double>(l[i]) - static_cast<double>(m)) : 0.0;
+                z += s[i];
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = i * 32 + lane;
+                s[i] = e < E ? 1.0 / (1.0 + exp(-static_cast<double>(l[i]))) : 0.0;
+                z += s[i];
+            }
+        }
+        z = warp_sum_d(z);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] += s[i] / z;
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        if (e < E) wsum[warp * E + e] = acc[i];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        double v = 0.0;
+#pragma unroll
+        for (int w = 0; w < kStatWarps; ++w) v += wsum[w * E + e];
+        partial[static_cast<int64_t>(blockIdx.x) * E + e] = v;
+    }
+}
+
+__global__ void __launch_bounds__(kFinalThreads)
+balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_t* __restrict__ counts,
+                     int T, int E, int k, float* __restrict__ P, float* __restrict__ f,
+                     float* __restrict__ loss) {
+    __shared__ double prod[kFinalThreads];
+    pdl_wait();
+    pdl_trigger();
+    // each thread owns experts e = threadIdx.x + i * blockDim.x and keeps their f*P sum
+    double mine = 0.0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        double sum = 0.0;
+        for (int c = 0; c < tiles; ++c) sum += partial[static_cast<int64_t>(c) * E + e];
+        const double Pe = T > 0 ? sum / T : 0.0;
+        const double fe = T > 0 ? static_cast<double>(E) * counts[e] / (static_cast<double>(k) * T) : 0.0;
+        P[e] = static_cast<float>(Pe);
+        f[e] = static_cast<float>(fe);
+        mine += fe * Pe;
+    }
+    prod[threadIdx.x] = mine;
+    __syncthreads();
+    for (int half = blockDim.x / 2; half > 0; half >>= 1) {  // fixed-order pairwise tree
+        if (threadIdx.x < half) prod[threadIdx.x] += prod[threadIdx.x + half];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *loss = static_cast<float>(prod[0]);
+}
+
+template <int EPL>
+cudaError_t launch_partial(const float* logits, int T, int E, int score_fn, double* partial,
+                           int tiles, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(kStatWarps) * E * sizeof(double);
+    static bool configured = false;
+    if (!configured && smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(balance_partial_kernel<EPL>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kStatWarps * TK_MAX_EXPERTS * static_cast<int>(sizeof(double)));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    return launch_pdl(balance_partial_kernel<EPL>, dim3(tiles), dim3(kStatWarps * 32), smem, s,
+                      logits, T, E, score_fn, partial);
+}
+
+__global__ void tp_mask_kernel(const int32_t* __restrict__ in, int64_t n, int lo, int el,
+                               int32_t* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int e = in[i];
+        out[i] = (e >= lo && e < lo + el) ? e - lo : -1;
+    }
+}
+
+int stat_tiles(int T) { return (T + kStatTileTokens - 1) / kStatTileTokens; }
+
+}  // namespace
+}  // namespace tk
+
+extern "C" size_t tk_balance_stats_workspace_bytes(int T, int E) {
+    if (T < 0 || E < 1) return 0;
+    const int tiles = tk::stat_tiles(T) > 0 ? tk::stat_tiles(T) : 1;
+    return static_cast<size_t>(tiles) * static_cast<size_t>(E) * sizeof(double);
+}
+
+extern "C" tk_status tk_balance_stats(const float* logits, const int32_t* counts, int T, int E,
+                                      int k, int score_fn, float* P, float* f, float* loss,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_balance_stats: T=%d must be >= 0", T);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_balance_stats: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (k < 1 || k > E || k > TK_MAX_TOPK)
+        return fail_arg("tk_balance_stats: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (score_fn != TK_SCORE_SOFTMAX && score_fn != TK_SCORE_SIGMOID)
+        return fail_arg("tk_balance_stats: unknown score_fn %d", score_fn);
+    if (counts == nullptr || P == nullptr || f == nullptr || loss == nullptr || workspace == nullptr)
+        return fail_arg("tk_balance_stats: counts, P, f, loss and workspace must not be NULL");
+    if (T > 0 && logits == nullptr) return fail_arg("tk_balance_stats: logits must not be NULL");
+    const size_t need = tk_balance_stats_workspace_bytes(T, E);
+    if (workspace_bytes < need)
+        return fail_arg("tk_balance_stats: workspace holds %zu bytes, needs %zu", workspace_bytes, need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+        return fail_arg("tk_balance_stats: workspace must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    double* partial = static_cast<double*>(workspace);
+    const int tiles = stat_tiles(T);
+    cudaError_t err = cudaSuccess;
+    if (tiles > 0) {
+        const int epl = (E + 31) / 32;
+        if (epl <= 1) err = launch_partial<1>(logits, T, E, score_fn, partial, tiles, s);
+        else if (epl <= 2) err = launch_partial<2>(logits, T, E, score_fn, partial, tiles, s);
+        else if (epl <= 4) err = launch_partial<4>(logits, T, E, score_fn, partial, tiles, s);
+        else if (epl <= 8) err = launch_partial<8>(logits, T, E, score_fn, partial, tiles, s);
+        else if (epl <= 16) err = launch_partial<16>(logits, T, E, score_fn, partial, tiles, s);
+        else err = launch_partial<32>(logits, T, E, score_fn, partial, tiles, s);
+        if (err != cudaSuccess) return check_launch(err, "balance_partial_kernel");
+    }
+    err = launch_pdl(balance_final_kernel, dim3(1), dim3(kFinalThreads), 0, s,
+                     static_cast<const double*>(partial), tiles, counts, T, E, k, P, f, loss);
+    return check_launch(err, "balance_final_kernel");
+}
+
+extern "C" tk_status tk_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size,
+                                int tp_rank, int32_t* out_idx, void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_tp_mask: T=%d must be >= 0", T);
+    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("tk_tp_mask: k=%d outside [1, %d]", k, TK_MAX_TOPK);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_tp_mask: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (tp_size < 1 || E % tp_size != 0)
+        return fail_arg("tk_tp_mask: tp_size=%d must divide E=%d", tp_size, E);
+    if (tp_rank < 0 || tp_rank >= tp_size)
+        return fail_arg("tk_tp_mask: tp_rank=%d outside [0, %d)", tp_rank, tp_size);
+    if (T == 0) return TK_OK;
+    if (topk_idx == nullptr || out_idx == nullptr) return fail_arg("tk_tp_mask: NULL pointer");
+    const int el = E / tp_size;
+    const int64_t n = static_cast<int64_t>(T) * k;
+    int64_t grid = (n + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+    if (grid > cap) grid = cap;
+    const cudaError_t err = launch_pdl(tp_mask_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                                       static_cast<cudaStream_t>(stream), topk_idx, n, tp_rank * el,
+                                       el, out_idx);
+    return check_launch(err, "tp_mask_kernel");
+}

@@ -26,7 +26,6 @@ namespace {
 constexpr uint32_t kCopyChunkBytes = 32768;  // bf16 bytes staged per bulk load
 constexpr int kFp8Threads = 256;
 constexpr int kFp8ChunkChannels = 8192;      // channels quantised per stage
-constexpr int kPadThreads = 256;
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
 
@@ -173,47 +172,6 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
     if (tid == 0) bulk_wait_read_all();
 }
 
-// Zeroes padding rows: rows r < offsets[E] with token_of[r] == -1. Padding comes in runs of up
-// to align-1 rows at the end of each expert's segment, so rows are dealt out round-robin over
-// CTAs (row r goes to CTA r % gridDim.x) to spread every run over many SMs. A thread that finds
-// a padding row enqueues bulk stores of a zeroed shared buffer over it (plus plain stores for
-// E4M3 scales), so the zeroing runs on the copy engines while the thread moves on.
-__global__ void __launch_bounds__(kPadThreads)
-expand_pad_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ token_of,
-                  int E, int64_t rmax, uint8_t* __restrict__ out, int64_t row_bytes,
-                  float* __restrict__ out_scale, int scale_cols, int32_t* err_flag) {
-    extern __shared__ __align__(128) uint8_t zeros[];  // min(row_bytes, kCopyChunkBytes)
-    const uint32_t zbytes = static_cast<uint32_t>(row_bytes < kCopyChunkBytes ? row_bytes : kCopyChunkBytes);
-    for (uint32_t o = threadIdx.x * 16u; o < zbytes; o += kPadThreads * 16u)
-        *reinterpret_cast<uint4*>(zeros + o) = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
-    __syncthreads();
-    pdl_wait();
-    pdl_trigger();
-    int64_t R = offsets[E];
-    if (R < 0 || R > rmax) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err_flag, TK_DEVERR_ROWS_RANGE);
-        R = R < 0 ? 0 : rmax;
-    }
-    bool issued = false;
-    for (int64_t r = blockIdx.x + static_cast<int64_t>(threadIdx.x) * gridDim.x; r < R;
-         r += static_cast<int64_t>(kPadThreads) * gridDim.x) {
-        if (token_of[r] != -1) continue;
-        uint8_t* row = out + r * row_bytes;
-        for (int64_t o = 0; o < row_bytes; o += zbytes) {
-            const int64_t left = row_bytes - o;
-            bulk_store(row + o, zeros, static_cast<uint32_t>(left < zbytes ? left : zbytes));
-        }
-        issued = true;
-        if (out_scale != nullptr)
-            for (int c = 0; c < scale_cols; ++c) out_scale[r * scale_cols + c] = 0.0f;
-    }
-    if (issued) {
-        bulk_commit();
-        bulk_wait_read_all();  // the shared zero buffer must outlive the stores that read it
-    }
-}
-
 }  // namespace
 }  // namespace tk
 
@@ -264,15 +222,10 @@ extern "C" tk_status tk_expand(const void* x, const int32_t* slot_of, const int3
     }
     if (align > 1) {
         const bool fp8 = out_dtype == TK_OUT_FP8_E4M3;
-        const int64_t row_bytes = fp8 ? H : static_cast<int64_t>(H) * 2;
-        int64_t grid = (rmax + kPadThreads - 1) / kPadThreads;
-        const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
-        if (grid > cap) grid = cap;
-        if (grid < 1) grid = 1;
-        const size_t zsmem = static_cast<size_t>(row_bytes < kCopyChunkBytes ? row_bytes : kCopyChunkBytes);
-        err = launch_pdl(expand_pad_kernel, dim3(static_cast<unsigned>(grid)), dim3(kPadThreads), zsmem, s,
-                         offsets, token_of, E, rmax, static_cast<uint8_t*>(out), row_bytes,
-                         fp8 ? out_scale : static_cast<float*>(nullptr), fp8 ? H / 128 : 0, err_flag);
+        err = launch_pad_zero(offsets, token_of, E, rmax, static_cast<uint8_t*>(out),
+                              fp8 ? H : static_cast<int64_t>(H) * 2,
+                              fp8 ? out_scale : static_cast<float*>(nullptr), fp8 ? H / 128 : 0,
+                              err_flag, s);
         if (err != cudaSuccess) return check_launch(err, "expand_pad_kernel");
     }
     return TK_OK;

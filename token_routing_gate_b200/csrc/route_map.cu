@@ -69,8 +69,8 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
         const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
         if (p >= p1) continue;
         const int e = e_reg[i];
-        if (e < 0 || e >= E) {
-            flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
+        if (e < 0 || e >= E) {  // -1 is a masked pair (tk_tp_mask), anything else an error
+            if (e != -1) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
             continue;
         }
         atomicAdd(&cnt[e], 1);  // integer counts: the order of the additions does not matter

@@ -38,6 +38,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Zeroes the padding rows of an expert-sorted buffer (rows r < offsets[E] with token_of[r] ==
+// -1): row_bytes per row, and scale_cols fp32 scales per row when out_scale is given.
+cudaError_t launch_pad_zero(const int32_t* offsets, const int32_t* token_of, int E, int64_t rmax,
+                            uint8_t* out, int64_t row_bytes, float* out_scale, int scale_cols,
+                            int32_t* err_flag, cudaStream_t s);
+
 // ------------------------------------------------------------------ device-side helpers
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

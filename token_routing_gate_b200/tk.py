@@ -25,7 +25,9 @@ DEVERR_TIMEOUT = 16
 
 # every C entry point declared in include/tk_route.h
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
-               "tk_route_map_static", "tk_expand", "tk_reduce", "tk_status_str",
+               "tk_route_map_static", "tk_expand", "tk_reduce", "tk_balance_stats_workspace_bytes",
+               "tk_balance_stats", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
+               "tk_reduce_backward", "tk_expand_backward", "tk_status_str",
                "tk_last_error_detail", "tk_abi_version")
 
 
@@ -57,6 +59,19 @@ def _load():
     L.tk_expand.restype = i32
     L.tk_reduce.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp, vp, vp]
     L.tk_reduce.restype = i32
+    L.tk_balance_stats_workspace_bytes.argtypes = [i32, i32]
+    L.tk_balance_stats_workspace_bytes.restype = sz
+    L.tk_balance_stats.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+    L.tk_balance_stats.restype = i32
+    L.tk_tp_mask.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp]
+    L.tk_tp_mask.restype = i32
+    L.tk_reduce_backward_workspace_bytes.argtypes = [i32, i32]
+    L.tk_reduce_backward_workspace_bytes.restype = sz
+    L.tk_reduce_backward.argtypes = [vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, sz,
+                                     vp, vp]
+    L.tk_reduce_backward.restype = i32
+    L.tk_expand_backward.argtypes = [vp, i64, vp, i32, i32, i32, vp, vp, vp]
+    L.tk_expand_backward.restype = i32
     L.tk_status_str.argtypes = [i32]
     L.tk_status_str.restype = ctypes.c_char_p
     L.tk_last_error_detail.argtypes = []
@@ -159,4 +174,68 @@ def reduce(y, slot_of, w=None, out=None, err_flag=None, stream=None):
         out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device)
     _check("tk_reduce", lib.tk_reduce(_ptr(y), y.shape[0], _ptr(slot_of), _ptr(w), T, k, H,
                                       _ptr(out), _ptr(err_flag), _stream(stream)))
+    return out
+
+
+def _workspace(nbytes, device):
+    return torch.empty((max(nbytes, 16) + 15) // 16, 16, dtype=torch.uint8, device=device)
+
+
+def balance_stats(logits, counts, k, score="sigmoid", workspace=None, out=None, stream=None):
+    """Load-balance statistics -> (P fp32 [E], f fp32 [E], loss fp32 [1])."""
+    T, E = logits.shape
+    dev = counts.device
+    if workspace is None:
+        workspace = _workspace(int(lib.tk_balance_stats_workspace_bytes(T, E)), dev)
+    if out is None:
+        out = (torch.empty(E, dtype=torch.float32, device=dev),
+               torch.empty(E, dtype=torch.float32, device=dev),
+               torch.empty(1, dtype=torch.float32, device=dev))
+    P, f, loss = out
+    _check("tk_balance_stats", lib.tk_balance_stats(
+        _ptr(logits), _ptr(counts), T, E, k, SCORE[score], _ptr(P), _ptr(f), _ptr(loss),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return P, f, loss
+
+
+def tp_mask(topk_idx, E, tp_size, tp_rank, out=None, stream=None):
+    """Keep this rank's experts (renumbered locally), mark the rest -1."""
+    T, k = topk_idx.shape
+    if out is None:
+        out = torch.empty_like(topk_idx)
+    _check("tk_tp_mask", lib.tk_tp_mask(_ptr(topk_idx), T, k, E, tp_size, tp_rank, _ptr(out),
+                                        _stream(stream)))
+    return out
+
+
+def reduce_backward(grad_out, y, slot_of, w, E, rm=None, d_y=None, d_w=None, workspace=None,
+                    err_flag=None, stream=None):
+    """Backward of reduce -> (d_y bf16 [rows, H], d_w fp32 [T, k]). With a RouteMap `rm`,
+    padding rows of d_y are zeroed."""
+    T, k = slot_of.shape
+    H = grad_out.shape[1]
+    dev = grad_out.device
+    if d_y is None:
+        d_y = torch.empty_like(y)
+    if d_w is None:
+        d_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _workspace(int(lib.tk_reduce_backward_workspace_bytes(T, k)), dev)
+    _check("tk_reduce_backward", lib.tk_reduce_backward(
+        _ptr(grad_out), _ptr(y), y.shape[0], _ptr(slot_of),
+        _ptr(rm.offsets) if rm is not None else None, _ptr(rm.token_of) if rm is not None else None,
+        _ptr(w), T, E, k, H, _ptr(d_y), _ptr(d_w), _ptr(workspace), workspace.numel(),
+        _ptr(err_flag), _stream(stream)))
+    return d_y, d_w
+
+
+def expand_backward(d_xe, slot_of, out=None, err_flag=None, stream=None):
+    """Backward of a bf16 expand: d_x[t] = sum_j d_xe[slot_of[t, j]]."""
+    T, k = slot_of.shape
+    H = d_xe.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=d_xe.device)
+    _check("tk_expand_backward", lib.tk_expand_backward(
+        _ptr(d_xe), d_xe.shape[0], _ptr(slot_of), T, k, H, _ptr(out), _ptr(err_flag),
+        _stream(stream)))
     return out
