@@ -42,6 +42,9 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for cpu_baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--op", choices=["step", "backward", "stats"], default="step",
+                   help="step: the forward path (the benchmark's headline); backward: reduce and "
+                        "expand backward; stats: load-balance statistics and the TP mask")
     return p.parse_args()
 
 
@@ -395,6 +398,72 @@ def run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out, 
             "ms_per_step": 1e3 * max_s / n}
 
 
+def run_op(args, wl):
+    """Time one of the next-row ops on the workload (single GPU), one JSON line."""
+    import torch
+    from token_routing_gate_b200 import tk
+    from token_routing_gate_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    logits, bias = W.gate_inputs(wl, dev)
+    idx, w = tk.gate_topk(logits, wl.k, wl.score, bias)
+    rm = tk.route_map(idx, wl.E, wl.align)
+    T, E, k, H = wl.T, wl.E, wl.k, wl.H
+    R = int(rm.offsets[-1].item())
+    if args.op == "backward":
+        y = W.expert_outputs(wl, dev)
+        g = W.activations(wl.with_(seed=wl.seed + 7), dev)
+        d_y = torch.empty_like(y)
+        d_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        ws = tk._workspace(int(tk.lib.tk_reduce_backward_workspace_bytes(T, k)), dev)
+        d_x = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        pad = (R - T * k) * H * 2 + (R * 4 if wl.align > 1 else 0)
+        calls = {
+            "reduce_backward": (lambda: tk.reduce_backward(g, y, rm.slot_of, w, E, rm=rm, d_y=d_y, d_w=d_w,
+                                                           workspace=ws, stream=stream),
+                                T * H * 2 + 2 * T * k * H * 2 + T * k * (8 + 4 + 64) + pad),
+            "expand_backward": (lambda: tk.expand_backward(d_y, rm.slot_of, out=d_x, stream=stream),
+                                T * k * H * 2 + T * k * 4 + T * H * 2),
+        }
+        metric = "reduce + expand backward HBM GB/s vs peak"
+    else:
+        P = (torch.empty(E, device=dev), torch.empty(E, device=dev), torch.empty(1, device=dev))
+        ws = tk._workspace(int(tk.lib.tk_balance_stats_workspace_bytes(T, E)), dev)
+        masked = torch.empty_like(idx)
+        calls = {
+            "balance_stats": (lambda: tk.balance_stats(logits, rm.counts, k, wl.score, workspace=ws, out=P,
+                                                       stream=stream),
+                              T * E * 4 + E * 4 + ((T + 63) // 64) * E * 8 * 2 + 3 * E * 4),
+            "tp_mask": (lambda: tk.tp_mask(idx, E, 8, 3, out=masked, stream=stream), T * k * 8),
+        }
+        metric = "load-balance statistics and TP mask us per call"
+    peak, peak_kind = load_peak()
+    out = {}
+    for name, (fn, nbytes) in calls.items():
+        for _ in range(args.warmup):
+            fn()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize(dev)
+        ev[0].record(stream)
+        for _ in range(args.steps):
+            fn()
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+        us = ev[0].elapsed_time(ev[1]) * 1e3 / args.steps
+        out[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak}
+    first = next(iter(out))
+    line = {"metric": metric, "op": args.op, "value": out[first]["gbs"] if args.op == "backward" else out[first]["us"],
+            "unit": "GB/s" if args.op == "backward" else "us", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": args.op == "backward", "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": wl.name, "T": T, "E": E, "k": k, "H": H,
+                                             "align": wl.align, "rows_used": R},
+            "peak": peak, "peak_kind": peak_kind, "kernels": out, "gpu_launches": None}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     from token_routing_gate_b200 import workloads as W
@@ -403,6 +472,8 @@ def main():
         wl = wl.with_(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.op != "step":
+        return run_op(args, wl)
     return run_tk(args, wl)
 
 

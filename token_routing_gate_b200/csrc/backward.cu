@@ -28,6 +28,7 @@ constexpr int kBwdThreads = 32 * (1 + kConsumerWarps);
 constexpr int kChunkCh = 8 * 32 * kConsumerWarps;  // channels per unit, one vector per thread
 constexpr int kChunkBytes = kChunkCh * 2;
 constexpr int kStageBudget = 40 * 1024;
+constexpr int kRegRows = 8;  // up to this k, per-thread register accumulators for d_w
 
 struct StageMeta {
     float w[TK_MAX_TOPK];
@@ -128,6 +129,13 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
         // ---------------- consumers
         const int ct = threadIdx.x - 32;
         const int cw = warp - 1;
+        // k <= 8: each thread keeps its partial dot product of every row in registers for the
+        // whole token and the warp reduces once per token; larger k reduces every chunk into
+        // per-warp shared accumulators.
+        const bool reg_acc = k <= kRegRows;
+        double accd[kRegRows];
+#pragma unroll
+        for (int j = 0; j < kRegRows; ++j) accd[j] = 0.0;
         int it = 0;
         for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
             for (int c = 0; c < chunks; ++c, ++it) {
@@ -141,42 +149,84 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
                 const int chn = min(kChunkCh, H - ch0);
                 const bool live = ct * 8 < chn;
                 const uint8_t* base = data + static_cast<size_t>(s) * stage_bytes + ct * 16;
+                uint8_t* dy_base = d_y + static_cast<int64_t>(ch0 + ct * 8) * 2;
                 float gv[8];
                 if (live) {
                     const uint4 q = *reinterpret_cast<const uint4*>(base);
                     gv[0] = lo_bf16(q.x); gv[1] = hi_bf16(q.x); gv[2] = lo_bf16(q.y); gv[3] = hi_bf16(q.y);
                     gv[4] = lo_bf16(q.z); gv[5] = hi_bf16(q.z); gv[6] = lo_bf16(q.w); gv[7] = hi_bf16(q.w);
                 }
-                for (int j = 0; j < k; ++j) {
-                    const int32_t sl = meta[s].slot[j];
-                    if (sl < 0) continue;  // the same for the whole warp
-                    double part = 0.0;
-                    if (live) {
+                if (reg_acc) {
+                    double gd[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gd[e] = live ? static_cast<double>(gv[e]) : 0.0;
+#pragma unroll
+                    for (int j = 0; j < kRegRows; ++j) {
+                        if (j >= k) break;
+                        const int32_t sl = meta[s].slot[j];
+                        if (sl < 0 || !live) continue;
                         const float wj = meta[s].w[j];
                         const uint4 q = *reinterpret_cast<const uint4*>(base + (1 + j) * kChunkBytes);
-                        const float yv[8] = {lo_bf16(q.x), hi_bf16(q.x), lo_bf16(q.y), hi_bf16(q.y),
-                                             lo_bf16(q.z), hi_bf16(q.z), lo_bf16(q.w), hi_bf16(q.w)};
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) part += static_cast<double>(__fmul_rn(gv[e], yv[e]));
+                        accd[j] = fma(gd[0], static_cast<double>(lo_bf16(q.x)), accd[j]);
+                        accd[j] = fma(gd[1], static_cast<double>(hi_bf16(q.x)), accd[j]);
+                        accd[j] = fma(gd[2], static_cast<double>(lo_bf16(q.y)), accd[j]);
+                        accd[j] = fma(gd[3], static_cast<double>(hi_bf16(q.y)), accd[j]);
+                        accd[j] = fma(gd[4], static_cast<double>(lo_bf16(q.z)), accd[j]);
+                        accd[j] = fma(gd[5], static_cast<double>(hi_bf16(q.z)), accd[j]);
+                        accd[j] = fma(gd[6], static_cast<double>(lo_bf16(q.w)), accd[j]);
+                        accd[j] = fma(gd[7], static_cast<double>(hi_bf16(q.w)), accd[j]);
                         uint4 o;
                         o.x = pack_bf16x2(__fmul_rn(wj, gv[0]), __fmul_rn(wj, gv[1]));
                         o.y = pack_bf16x2(__fmul_rn(wj, gv[2]), __fmul_rn(wj, gv[3]));
                         o.z = pack_bf16x2(__fmul_rn(wj, gv[4]), __fmul_rn(wj, gv[5]));
                         o.w = pack_bf16x2(__fmul_rn(wj, gv[6]), __fmul_rn(wj, gv[7]));
-                        st_v4(d_y + static_cast<int64_t>(sl) * row_bytes + static_cast<int64_t>(ch0 + ct * 8) * 2, o);
+                        st_v4(dy_base + static_cast<int64_t>(sl) * row_bytes, o);
                     }
+                } else {
+                    for (int j = 0; j < k; ++j) {
+                        const int32_t sl = meta[s].slot[j];
+                        if (sl < 0) continue;  // the same for the whole warp
+                        double part = 0.0;
+                        if (live) {
+                            const float wj = meta[s].w[j];
+                            const uint4 q = *reinterpret_cast<const uint4*>(base + (1 + j) * kChunkBytes);
+                            const float yv[8] = {lo_bf16(q.x), hi_bf16(q.x), lo_bf16(q.y), hi_bf16(q.y),
+                                                 lo_bf16(q.z), hi_bf16(q.z), lo_bf16(q.w), hi_bf16(q.w)};
 #pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFullMask, part, off);
-                    if (lane == 0) dacc[cw * TK_MAX_TOPK + j] += part;
+                            for (int e = 0; e < 8; ++e)
+                                part = fma(static_cast<double>(gv[e]), static_cast<double>(yv[e]), part);
+                            uint4 o;
+                            o.x = pack_bf16x2(__fmul_rn(wj, gv[0]), __fmul_rn(wj, gv[1]));
+                            o.y = pack_bf16x2(__fmul_rn(wj, gv[2]), __fmul_rn(wj, gv[3]));
+                            o.z = pack_bf16x2(__fmul_rn(wj, gv[4]), __fmul_rn(wj, gv[5]));
+                            o.w = pack_bf16x2(__fmul_rn(wj, gv[6]), __fmul_rn(wj, gv[7]));
+                            st_v4(dy_base + static_cast<int64_t>(sl) * row_bytes, o);
+                        }
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFullMask, part, off);
+                        if (lane == 0) dacc[cw * TK_MAX_TOPK + j] += part;
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
                 if (c == chunks - 1) {  // token done: this warp's sums go out, accumulators reset
-                    if (lane < k) {
-                        dw_part[(t * k + lane) * kConsumerWarps + cw] = dacc[cw * TK_MAX_TOPK + lane];
-                        dacc[cw * TK_MAX_TOPK + lane] = 0.0;
+                    if (reg_acc) {
+#pragma unroll
+                        for (int j = 0; j < kRegRows; ++j) {
+                            if (j >= k) break;
+                            double v = accd[j];
+#pragma unroll
+                            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFullMask, v, off);
+                            if (lane == 0) dw_part[(t * k + j) * kConsumerWarps + cw] = v;
+                            accd[j] = 0.0;
+                        }
+                    } else {
+                        if (lane < k) {
+                            dw_part[(t * k + lane) * kConsumerWarps + cw] = dacc[cw * TK_MAX_TOPK + lane];
+                            dacc[cw * TK_MAX_TOPK + lane] = 0.0;
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
         }

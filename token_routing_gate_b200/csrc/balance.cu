@@ -80,9 +80,9 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
                 z += s[i];
             }
         }
-        z = warp_sum_d(z);
+        const double rz = 1.0 / warp_sum_d(z);
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) acc[i] += s[i] / z;
+        for (int i = 0; i < EPL; ++i) acc[i] += s[i] * rz;
     }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
