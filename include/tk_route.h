@@ -24,9 +24,9 @@
  *    a buffer) never fault: the kernel skips the offending element and ORs a TK_DEVERR_* bit
  *    into *err_flag when err_flag (a device int32, nullable) is given. The caller zeroes
  *    *err_flag beforehand and reads it after synchronising the stream.
- *  - Kernels launch with programmatic dependent launch enabled: each kernel may be scheduled
- *    while the previous kernel on the stream finishes, but reads no input before that kernel
- *    has completed.
+ *  - Kernels launch with programmatic dependent launch enabled (the launch latency of a kernel
+ *    overlaps the end of the previous one); no kernel reads an input before the previous
+ *    kernel on the stream has completed.
  */
 #ifndef TK_ROUTE_H
 #define TK_ROUTE_H

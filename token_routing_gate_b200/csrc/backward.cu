@@ -79,7 +79,6 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
     for (int i = threadIdx.x; i < kConsumerWarps * TK_MAX_TOPK; i += blockDim.x) dacc[i] = 0.0;
     __syncthreads();
     pdl_wait();
-    pdl_trigger();
 
     const int chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t row_bytes = static_cast<int64_t>(H) * 2;
@@ -236,7 +235,6 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
 __global__ void dw_combine_kernel(const double* __restrict__ dw_part, int64_t pairs,
                                   float* __restrict__ d_w) {
     pdl_wait();
-    pdl_trigger();
     for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; p < pairs;
          p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         double v = 0.0;

@@ -42,7 +42,6 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
                        double* __restrict__ partial) {
     extern __shared__ double wsum[];  // [kStatWarps][E]
     pdl_wait();
-    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     double acc[EPL];
@@ -104,7 +103,6 @@ balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_
                      float* __restrict__ loss) {
     __shared__ double prod[kFinalThreads];
     pdl_wait();
-    pdl_trigger();
     // each thread owns experts e = threadIdx.x + i * blockDim.x and keeps their f*P sum
     double mine = 0.0;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -144,7 +142,6 @@ cudaError_t launch_partial(const float* logits, int T, int E, int score_fn, doub
 __global__ void tp_mask_kernel(const int32_t* __restrict__ in, int64_t n, int lo, int el,
                                int32_t* __restrict__ out) {
     pdl_wait();
-    pdl_trigger();
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int e = in[i];

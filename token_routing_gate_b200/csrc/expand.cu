@@ -43,7 +43,6 @@ expand_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ sl
     }
     __syncwarp();
     pdl_wait();
-    pdl_trigger();
     int64_t my_slot = -1;
     if (lane < k) {
         const int64_t s = slot_of[t * k + lane];
@@ -102,7 +101,6 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
     }
     __syncthreads();
     pdl_wait();
-    pdl_trigger();
     if (tid < k) {
         const int64_t s = slot_of[t * k + tid];
         int64_t v = -1;

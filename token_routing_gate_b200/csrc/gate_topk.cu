@@ -100,7 +100,6 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
                  int k, int score_fn, int renormalize, int tokens_per_warp,
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     pdl_wait();
-    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t t_begin = (static_cast<int64_t>(blockIdx.x) * kGateWarps + (threadIdx.x >> 5)) * tokens_per_warp;
     if (t_begin >= T) return;

@@ -28,7 +28,6 @@ expand_pad_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict
     fence_proxy_async_smem();
     __syncthreads();
     pdl_wait();
-    pdl_trigger();
     int64_t R = offsets[E];
     if (R < 0 || R > rmax) {
         if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(err_flag, TK_DEVERR_ROWS_RANGE);

@@ -95,7 +95,6 @@ reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __re
     }
     __syncthreads();
     pdl_wait();
-    pdl_trigger();
 
     const int chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t units = static_cast<int64_t>(T) * chunks;

@@ -45,7 +45,6 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
                    int64_t rmax, int32_t* err_flag) {
     extern __shared__ int32_t cnt[];  // [E]
     pdl_wait();
-    pdl_trigger();
     const int tile = blockIdx.x;
     const int64_t p0 = static_cast<int64_t>(tile) * kTileTokens * k;
     const int64_t p1 = min(static_cast<int64_t>(T), static_cast<int64_t>(tile + 1) * kTileTokens) * k;
@@ -89,7 +88,6 @@ route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align
     __shared__ int32_t warp_tot[kScanThreads / 32];
     __shared__ int32_t carry;
     pdl_wait();
-    pdl_trigger();
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31;
@@ -154,7 +152,6 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     uint32_t* bitmap = smem;                                          // [E][kTileWords]
     int32_t* base = reinterpret_cast<int32_t*>(smem + E * kTileWords);  // [E]
     pdl_wait();
-    pdl_trigger();
     const int tile = blockIdx.x;
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
@@ -219,7 +216,6 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
     __shared__ int32_t warp_tot[kRouteThreads / 32];
     __shared__ int32_t carry;
     pdl_wait();
-    pdl_trigger();
     const int tile = blockIdx.x;
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
