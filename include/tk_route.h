@@ -225,6 +225,15 @@ TK_API tk_status tk_expand_backward(const void* d_xe, int64_t xe_rows, const int
                                     int T, int k, int H, void* d_x, int32_t* err_flag,
                                     void* stream);
 
+/*
+ * Self-test of the library's bounded waits (no counterpart on the pages: it exists so that the
+ * failure path can be exercised without faulting a GPU). One warp waits on an mbarrier that
+ * nothing ever completes, using the same bounded wait as every kernel here; after limit_ns
+ * nanoseconds (1 .. 2e9) the wait gives up, TK_DEVERR_TIMEOUT is ORed into *err_flag (device
+ * int32) and the kernel returns, leaving the context usable.
+ */
+TK_API tk_status tk_selftest_bounded_wait(int64_t limit_ns, int32_t* err_flag, void* stream);
+
 /* Name of a status code (static string). */
 TK_API const char* tk_status_str(int status);
 

@@ -163,3 +163,9 @@ def test_next_rows_reject_bad_arguments(tk):
         assert L.tk_reduce_backward(*a) == 1, what
         assert what in L.tk_last_error_detail().decode()
     assert L.tk_expand_backward(FAKE, 10, FAKE, 4, 0, 256, FAKE, None, None) == 1
+
+
+def test_selftest_rejects_bad_limits(tk):
+    assert tk.lib.tk_selftest_bounded_wait(0, FAKE, None) == 1
+    assert tk.lib.tk_selftest_bounded_wait(3_000_000_000, FAKE, None) == 1
+    assert tk.lib.tk_selftest_bounded_wait(1000, None, None) == 1

@@ -100,3 +100,21 @@ def test_host_errors_raise_before_launch():
         tk.reduce(x, torch.zeros(4, 2, dtype=torch.int32, device="cuda"))
     with pytest.raises(tk.TkError, match="bias"):
         tk.gate_topk(torch.zeros(4, 8, device="cuda"), 2, "softmax", torch.zeros(8, device="cuda"))
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    import time
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    tk.selftest_bounded_wait(20_000_000, err)          # 20 ms on a barrier nothing completes
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert err.item() == tk.DEVERR_TIMEOUT
+    assert 0.015 < dt < 5.0
+    # the context still works: a full routing step right after
+    x = torch.randn(64, 256, device="cuda").to(torch.bfloat16)
+    idx, w = tk.gate_topk(torch.randn(64, 16, device="cuda"), 2, "sigmoid")
+    rm = tk.route_map(idx, 16)
+    out = tk.reduce(tk.expand(x, rm, 16, 2), rm.slot_of, None)
+    torch.cuda.synchronize()
+    assert torch.equal(out.float(), (2 * x.float()).to(torch.bfloat16).float())

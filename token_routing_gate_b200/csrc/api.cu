@@ -44,7 +44,35 @@ int num_sms() {
     return cached[dev];
 }
 
+namespace {
+
+// Waits on an mbarrier that nothing ever arrives on, with the library's bounded wait: the wait
+// must give up after limit_ns, flag TK_DEVERR_TIMEOUT and let the kernel return normally.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int32_t* err_flag) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (!mbar_wait_bounded(&bar, 0, limit_ns)) {
+        if (threadIdx.x == 0) flag_error(err_flag, TK_DEVERR_TIMEOUT);
+    }
+}
+
+}  // namespace
 }  // namespace tk
+
+extern "C" tk_status tk_selftest_bounded_wait(int64_t limit_ns, int32_t* err_flag, void* stream) {
+    using namespace tk;
+    if (limit_ns < 1 || limit_ns > INT64_C(2000000000))
+        return fail_arg("tk_selftest_bounded_wait: limit_ns=%lld outside [1, 2e9]", (long long)limit_ns);
+    if (err_flag == nullptr) return fail_arg("tk_selftest_bounded_wait: err_flag must not be NULL");
+    const cudaError_t err = launch_pdl(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0,
+                                       static_cast<cudaStream_t>(stream),
+                                       static_cast<uint64_t>(limit_ns), err_flag);
+    return check_launch(err, "bounded_wait_selftest_kernel");
+}
 
 extern "C" const char* tk_status_str(int status) {
     switch (status) {

@@ -81,6 +81,96 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     }
 }
 
+// ---- rank phase shared by every scatter variant: bitmap of the tile's tokens per expert, then
+// slot = base[e] + (number of the tile's earlier tokens on expert e)
+__device__ __forceinline__ void tile_mark(uint32_t* bitmap, const int (&e_reg)[kPairsPerThread],
+                                          int iters, int64_t p0, int64_t p1, int k, int t0, int E,
+                                          int32_t* err_flag) {
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        const int e = e_reg[i];
+        if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged elsewhere
+        const int tl = static_cast<int>(p / k) - t0;
+        const uint32_t bit = 1u << (tl & 31);
+        const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
+        if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
+    }
+}
+
+__device__ __forceinline__ void tile_scatter(const uint32_t* bitmap, const int32_t* base,
+                                             const int (&e_reg)[kPairsPerThread], int iters,
+                                             int64_t p0, int64_t p1, int k, int t0, int E,
+                                             int32_t* slot_of, int32_t* token_of) {
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= iters) break;
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        if (p >= p1) continue;
+        const int e = e_reg[i];
+        if (e < 0 || e >= E) {
+            slot_of[p] = -1;
+            continue;
+        }
+        const int t = static_cast<int>(p / k);
+        const int tl = t - t0;
+        const uint32_t* bm = bitmap + e * kTileWords;
+        int rank = __popc(bm[tl >> 5] & ((1u << (tl & 31)) - 1u));
+        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bm[w]);
+        const int32_t slot = base[e] + rank;
+        slot_of[p] = slot;
+        token_of[slot] = t;
+    }
+}
+
+__device__ __forceinline__ int load_tile(const int32_t* topk_idx, int64_t p0, int64_t p1,
+                                         int (&e_reg)[kPairsPerThread]) {
+    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
+    }
+    return iters;
+}
+
+// Exclusive scan of ceil(total[e]/align)*align over experts, for a whole CTA of kRouteThreads
+// threads: writes excl[e] (the segment offset of expert e) and returns the grand total R.
+__device__ __forceinline__ int32_t cta_padded_scan(const int32_t* total, int E, int align,
+                                                   int32_t* excl, int32_t* warp_tot) {
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    int32_t carry = 0;
+    for (int e0 = 0; e0 < E; e0 += kRouteThreads) {
+        const int e = e0 + threadIdx.x;
+        const int32_t padded = e < E ? (total[e] + align - 1) / align * align : 0;
+        int32_t incl = padded;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t u = __shfl_up_sync(kFullMask, incl, off);
+            if (lane >= off) incl += u;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            constexpr int nw = kRouteThreads / 32;
+            int32_t u = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int32_t q = __shfl_up_sync(kFullMask, u, off);
+                if (lane >= off) u += q;
+            }
+            if (lane < nw) warp_tot[lane] = u;
+        }
+        __syncthreads();
+        if (e < E) excl[e] = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + incl - padded;
+        carry += warp_tot[kRouteThreads / 32 - 1];
+        __syncthreads();
+    }
+    return carry;
+}
+
 // Single CTA. Column e of tile_counts becomes exclusive per-tile prefixes (in place).
 __global__ void __launch_bounds__(kScanThreads)
 route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align,
@@ -156,167 +246,72 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
     const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
-    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
     int e_reg[kPairsPerThread];
-#pragma unroll
-    for (int i = 0; i < kPairsPerThread; ++i) {
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
-    }
+    const int iters = load_tile(topk_idx, p0, p1, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     for (int e = threadIdx.x; e < E; e += kRouteThreads)
         base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(tile) * E + e];
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        const int e = e_reg[i];
-        if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged by the count kernel
-        const int tl = static_cast<int>(p / k) - t0;
-        const uint32_t bit = 1u << (tl & 31);
-        const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
-        if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
-    }
+    tile_mark(bitmap, e_reg, iters, p0, p1, k, t0, E, err_flag);
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        if (p >= p1) continue;
-        const int e = e_reg[i];
-        if (e < 0 || e >= E) {
-            slot_of[p] = -1;
-            continue;
-        }
-        const int t = static_cast<int>(p / k);
-        const int tl = t - t0;
-        const uint32_t* bm = bitmap + e * kTileWords;
-        int rank = __popc(bm[tl >> 5] & ((1u << (tl & 31)) - 1u));
-        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bm[w]);
-        const int32_t slot = base[e] + rank;
-        slot_of[p] = slot;
-        token_of[slot] = t;
-    }
+    tile_scatter(bitmap, base, e_reg, iters, p0, p1, k, t0, E, slot_of, token_of);
 }
 
 // Scan and scatter in one kernel, for batches of at most kFusedMaxTiles tiles: every CTA reads
 // the whole (small) count matrix itself -- its own tile's prefix per expert, and every column's
 // total for the offsets -- instead of waiting for a separate scan kernel. CTA 0 also writes
 // counts[] and offsets[]. The slot arithmetic is the same as route_scan + route_scatter.
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kRouteThreads, 1)
 route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int align,
                           const int32_t* __restrict__ tile_counts, int tiles,
                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                           int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
                           int32_t* err_flag) {
     extern __shared__ uint32_t smem[];
-    uint32_t* bitmap = smem;                                            // [E][kTileWords]
-    int32_t* base = reinterpret_cast<int32_t*>(smem + E * kTileWords);  // [E]
+    uint32_t* bitmap = smem;                                              // [E][kTileWords]
+    int32_t* before = reinterpret_cast<int32_t*>(bitmap + E * kTileWords);  // [E]
+    int32_t* total = before + E;                                          // [E]
+    int32_t* base = total + E;                                            // [E]
     __shared__ int32_t warp_tot[kRouteThreads / 32];
-    __shared__ int32_t carry;
     pdl_wait();
     const int tile = blockIdx.x;
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
     const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
-    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
     int e_reg[kPairsPerThread];
-#pragma unroll
-    for (int i = 0; i < kPairsPerThread; ++i) {
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
-    }
+    const int iters = load_tile(topk_idx, p0, p1, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
-    if (threadIdx.x == 0) carry = 0;
-    __syncthreads();
-
-    // ---- per expert: prefix over the tiles before this one, and the column total
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    for (int e0 = 0; e0 < E; e0 += kRouteThreads) {
-        const int e = e0 + threadIdx.x;
-        int32_t before = 0, total = 0;
-        if (e < E) {
-            for (int c0 = 0; c0 < tiles; c0 += kScanBatch) {
-                int32_t v[kScanBatch];
+    // per expert: the count over the tiles before this one, and the column total
+    for (int e = threadIdx.x; e < E; e += kRouteThreads) {
+        int32_t b = 0, tot = 0;
+        for (int c0 = 0; c0 < tiles; c0 += kScanBatch) {
+            int32_t v[kScanBatch];
 #pragma unroll
-                for (int i = 0; i < kScanBatch; ++i)
-                    v[i] = c0 + i < tiles ? tile_counts[static_cast<int64_t>(c0 + i) * E + e] : 0;
+            for (int i = 0; i < kScanBatch; ++i)
+                v[i] = c0 + i < tiles ? tile_counts[static_cast<int64_t>(c0 + i) * E + e] : 0;
 #pragma unroll
-                for (int i = 0; i < kScanBatch; ++i) {
-                    if (c0 + i < tile) before += v[i];
-                    total += v[i];
-                }
+            for (int i = 0; i < kScanBatch; ++i) {
+                if (c0 + i < tile) b += v[i];
+                tot += v[i];
             }
         }
-        const int32_t padded = e < E ? (total + align - 1) / align * align : 0;
-        int32_t incl = padded;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int32_t u = __shfl_up_sync(kFullMask, incl, off);
-            if (lane >= off) incl += u;
-        }
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            constexpr int nw = kRouteThreads / 32;
-            int32_t u = lane < nw ? warp_tot[lane] : 0;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int32_t q = __shfl_up_sync(kFullMask, u, off);
-                if (lane >= off) u += q;
-            }
-            if (lane < nw) warp_tot[lane] = u;
-        }
-        __syncthreads();
-        const int32_t excl = carry + (warp > 0 ? warp_tot[warp - 1] : 0) + incl - padded;
-        if (e < E) {
-            base[e] = excl + before;
-            if (tile == 0) {
-                counts[e] = total;
-                offsets[e] = excl;
-            }
-        }
-        const int32_t chunk_total = warp_tot[kRouteThreads / 32 - 1];
-        __syncthreads();
-        if (threadIdx.x == 0) carry += chunk_total;
-        __syncthreads();
-    }
-    if (tile == 0 && threadIdx.x == 0) offsets[E] = carry;
-
-    // ---- ranks inside the tile, as in route_scatter_kernel
-#pragma unroll
-    for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        const int e = e_reg[i];
-        if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged by the count kernel
-        const int tl = static_cast<int>(p / k) - t0;
-        const uint32_t bit = 1u << (tl & 31);
-        const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
-        if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
+        before[e] = b;
+        total[e] = tot;
     }
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        if (p >= p1) continue;
-        const int e = e_reg[i];
-        if (e < 0 || e >= E) {
-            slot_of[p] = -1;
-            continue;
+    const int32_t R = cta_padded_scan(total, E, align, base, warp_tot);
+    for (int e = threadIdx.x; e < E; e += kRouteThreads) {
+        if (tile == 0) {
+            counts[e] = total[e];
+            offsets[e] = base[e];
         }
-        const int t = static_cast<int>(p / k);
-        const int tl = t - t0;
-        const uint32_t* bm = bitmap + e * kTileWords;
-        int rank = __popc(bm[tl >> 5] & ((1u << (tl & 31)) - 1u));
-        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bm[w]);
-        const int32_t slot = base[e] + rank;
-        slot_of[p] = slot;
-        token_of[slot] = t;
+        base[e] += before[e];
     }
+    if (tile == 0 && threadIdx.x == 0) offsets[E] = R;
+    __syncthreads();
+    tile_mark(bitmap, e_reg, iters, p0, p1, k, t0, E, err_flag);
+    __syncthreads();
+    tile_scatter(bitmap, base, e_reg, iters, p0, p1, k, t0, E, slot_of, token_of);
 }
 
 }  // namespace
@@ -369,7 +364,7 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
                                  tile_counts, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
     if (tiles > 0 && tiles <= kFusedMaxTiles) {
-        const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
+        const size_t smem = static_cast<size_t>(E) * (kTileWords + 3) * sizeof(uint32_t);
         err = launch_pdl(route_scan_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s,
                          topk_idx, T, E, k, align, static_cast<const int32_t*>(tile_counts), tiles,
                          counts, offsets, slot_of, token_of, err_flag);

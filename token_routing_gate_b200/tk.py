@@ -27,7 +27,7 @@ DEVERR_TIMEOUT = 16
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
                "tk_route_map_static", "tk_expand", "tk_reduce", "tk_balance_stats_workspace_bytes",
                "tk_balance_stats", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
-               "tk_reduce_backward", "tk_expand_backward", "tk_status_str",
+               "tk_reduce_backward", "tk_expand_backward", "tk_selftest_bounded_wait", "tk_status_str",
                "tk_last_error_detail", "tk_abi_version")
 
 
@@ -72,6 +72,8 @@ def _load():
     L.tk_reduce_backward.restype = i32
     L.tk_expand_backward.argtypes = [vp, i64, vp, i32, i32, i32, vp, vp, vp]
     L.tk_expand_backward.restype = i32
+    L.tk_selftest_bounded_wait.argtypes = [i64, vp, vp]
+    L.tk_selftest_bounded_wait.restype = i32
     L.tk_status_str.argtypes = [i32]
     L.tk_status_str.restype = ctypes.c_char_p
     L.tk_last_error_detail.argtypes = []
@@ -239,3 +241,9 @@ def expand_backward(d_xe, slot_of, out=None, err_flag=None, stream=None):
         _ptr(d_xe), d_xe.shape[0], _ptr(slot_of), T, k, H, _ptr(out), _ptr(err_flag),
         _stream(stream)))
     return out
+
+
+def selftest_bounded_wait(limit_ns, err_flag, stream=None):
+    """Run the bounded-wait self-test kernel (it always times out and flags DEVERR_TIMEOUT)."""
+    _check("tk_selftest_bounded_wait", lib.tk_selftest_bounded_wait(int(limit_ns), _ptr(err_flag),
+                                                                    _stream(stream)))
