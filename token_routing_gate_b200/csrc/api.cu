@@ -32,16 +32,26 @@ tk_status check_launch(cudaError_t err, const char* what) {
     return TK_ERR_CUDA;
 }
 
-int num_sms() {
-    static int cached[64] = {0};
+int current_device() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (cached[dev] == 0) {
-        int n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+    return dev;
+}
+
+std::mutex& setup_mutex() {
+    static std::mutex m;
+    return m;
+}
+
+int num_sms() {
+    static std::atomic<int> cached[kMaxDevices];
+    const int dev = current_device();
+    int n = cached[dev].load(std::memory_order_acquire);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 1;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_release);
     }
-    return cached[dev];
+    return n;
 }
 
 namespace {

@@ -245,26 +245,38 @@ __global__ void dw_combine_kernel(const double* __restrict__ dw_part, int64_t pa
 }
 
 struct Shape {
-    int k = 0, S = 0, grid_cap = 0;
+    int S = 0, grid_cap = 0;
 };
 
-cudaError_t prepare(int k, Shape& sh) {
-    static int configured = 0;
-    const int S = stages_for(k);
-    const size_t smem = smem_bytes(k, S);
-    cudaError_t err = cudaSuccess;
-    if (static_cast<int>(smem) > configured) {
-        err = cudaFuncSetAttribute(reduce_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem));
-        if (err != cudaSuccess) return err;
-        configured = static_cast<int>(smem);
+// Launch shape for k on the current device, worked out once.
+cudaError_t launch_shape(int k, Shape& out) {
+    static Shape shapes[kMaxDevices][TK_MAX_TOPK + 1];
+    static std::atomic<bool> ready[kMaxDevices][TK_MAX_TOPK + 1];
+    static int configured[kMaxDevices];
+    const int dev = current_device();
+    if (ready[dev][k].load(std::memory_order_acquire)) {
+        out = shapes[dev][k];
+        return cudaSuccess;
     }
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_backward_kernel, kBwdThreads, smem);
-    if (err != cudaSuccess) return err;
-    sh.k = k;
-    sh.S = S;
-    sh.grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
+    std::lock_guard<std::mutex> lock(setup_mutex());
+    if (!ready[dev][k].load(std::memory_order_relaxed)) {
+        const int S = stages_for(k);
+        const size_t smem = smem_bytes(k, S);
+        cudaError_t err = cudaSuccess;
+        if (static_cast<int>(smem) > configured[dev]) {
+            err = cudaFuncSetAttribute(reduce_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+            if (err != cudaSuccess) return err;
+            configured[dev] = static_cast<int>(smem);
+        }
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_backward_kernel, kBwdThreads, smem);
+        if (err != cudaSuccess) return err;
+        shapes[dev][k].S = S;
+        shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
+        ready[dev][k].store(true, std::memory_order_release);
+    }
+    out = shapes[dev][k];
     return cudaSuccess;
 }
 
@@ -302,12 +314,9 @@ extern "C" tk_status tk_reduce_backward(const void* grad_out, const void* y, int
     const size_t need = tk_reduce_backward_workspace_bytes(T, k);
     if (workspace_bytes < need)
         return fail_arg("tk_reduce_backward: workspace holds %zu bytes, needs %zu", workspace_bytes, need);
-    static Shape shapes[TK_MAX_TOPK + 1];
-    Shape& sh = shapes[k];
-    if (sh.k != k) {
-        const cudaError_t e = prepare(k, sh);
-        if (e != cudaSuccess) return check_launch(e, "reduce_backward_kernel setup");
-    }
+    Shape sh;
+    const cudaError_t e = launch_shape(k, sh);
+    if (e != cudaSuccess) return check_launch(e, "reduce_backward_kernel setup");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     double* dw_part = static_cast<double*>(workspace);
     const int grid = T < sh.grid_cap ? T : sh.grid_cap;

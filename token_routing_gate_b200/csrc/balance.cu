@@ -127,13 +127,15 @@ template <int EPL>
 cudaError_t launch_partial(const float* logits, int T, int E, int score_fn, double* partial,
                            int tiles, cudaStream_t s) {
     const size_t smem = static_cast<size_t>(kStatWarps) * E * sizeof(double);
-    static bool configured = false;
-    if (!configured && smem > 48 * 1024) {
+    static std::atomic<bool> configured[kMaxDevices];
+    const int dev = current_device();
+    if (smem > 48 * 1024 && !configured[dev].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(setup_mutex());
         const cudaError_t e = cudaFuncSetAttribute(balance_partial_kernel<EPL>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    kStatWarps * TK_MAX_EXPERTS * static_cast<int>(sizeof(double)));
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     return launch_pdl(balance_partial_kernel<EPL>, dim3(tiles), dim3(kStatWarps * 32), smem, s,
                       logits, T, E, score_fn, partial);

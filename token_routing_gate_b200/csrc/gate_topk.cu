@@ -206,13 +206,16 @@ template <int EPL>
 cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, int k, int score_fn,
                         int renormalize, int32_t* idx, float* w, cudaStream_t s) {
     // one wave: as many warps as fit on the GPU at once, each taking consecutive tokens
-    static int resident_warps = 0;
+    static std::atomic<int> resident[kMaxDevices];
+    const int dev = current_device();
+    int resident_warps = resident[dev].load(std::memory_order_acquire);
     if (resident_warps == 0) {
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gate_topk_kernel<EPL>,
                                                           kGateWarps * 32, 0) != cudaSuccess || per_sm < 1)
             per_sm = 1;
         resident_warps = per_sm * kGateWarps * num_sms();
+        resident[dev].store(resident_warps, std::memory_order_release);
     }
     const int tpw = (T + resident_warps - 1) / resident_warps;
     const int warps = (T + tpw - 1) / tpw;

@@ -200,27 +200,38 @@ reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __re
 struct LaunchShape {
     int grid_cap = 0;   // SMs x resident CTAs for the current stage count
     int S = 0;
-    int k = 0;
 };
 
-cudaError_t prepare(int k, LaunchShape& shape) {
-    static int configured_smem = 0;
-    const int S = stages_for(k);
-    const size_t smem = smem_bytes(k, S);
-    cudaError_t err = cudaSuccess;
-    if (static_cast<int>(smem) > configured_smem) {
-        err = cudaFuncSetAttribute(reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem));
-        if (err != cudaSuccess) return err;
-        configured_smem = static_cast<int>(smem);
+// Launch shape for k on the current device, worked out once (the kernel's shared-memory limit
+// is raised to the largest size any k needs).
+cudaError_t launch_shape(int k, LaunchShape& out) {
+    static LaunchShape shapes[kMaxDevices][TK_MAX_TOPK + 1];
+    static std::atomic<bool> ready[kMaxDevices][TK_MAX_TOPK + 1];
+    static int configured_smem[kMaxDevices];
+    const int dev = current_device();
+    if (ready[dev][k].load(std::memory_order_acquire)) {
+        out = shapes[dev][k];
+        return cudaSuccess;
     }
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel, kRedThreads, smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
-    shape.grid_cap = num_sms() * per_sm;
-    shape.S = S;
-    shape.k = k;
+    std::lock_guard<std::mutex> lock(setup_mutex());
+    if (!ready[dev][k].load(std::memory_order_relaxed)) {
+        const int S = stages_for(k);
+        const size_t smem = smem_bytes(k, S);
+        cudaError_t err = cudaSuccess;
+        if (static_cast<int>(smem) > configured_smem[dev]) {
+            err = cudaFuncSetAttribute(reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+            if (err != cudaSuccess) return err;
+            configured_smem[dev] = static_cast<int>(smem);
+        }
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel, kRedThreads, smem);
+        if (err != cudaSuccess) return err;
+        shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
+        shapes[dev][k].S = S;
+        ready[dev][k].store(true, std::memory_order_release);
+    }
+    out = shapes[dev][k];
     return cudaSuccess;
 }
 
@@ -239,12 +250,9 @@ extern "C" tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slo
         return fail_arg("tk_reduce: y, slot_of and out must not be NULL");
     if (reinterpret_cast<uintptr_t>(y) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 16 != 0)
         return fail_arg("tk_reduce: y and out must be 16-byte aligned");
-    static LaunchShape shapes[TK_MAX_TOPK + 1];
-    LaunchShape& shape = shapes[k];
-    if (shape.k != k) {
-        const cudaError_t e = prepare(k, shape);
-        if (e != cudaSuccess) return check_launch(e, "reduce_kernel setup");
-    }
+    LaunchShape shape;
+    const cudaError_t e = launch_shape(k, shape);
+    if (e != cudaSuccess) return check_launch(e, "reduce_kernel setup");
     const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t units = static_cast<int64_t>(T) * chunks;
     const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);

@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "tk_route.h"
 
 namespace tk {
@@ -39,6 +42,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 int num_sms();  // SM count of the current device (cached per device)
+
+// Launch shapes (occupancy, shared-memory opt-in) are worked out once per device on the first
+// call and cached: current_device() indexes the caches, setup_mutex() serialises their filling.
+constexpr int kMaxDevices = 64;
+int current_device();
+std::mutex& setup_mutex();
 
 // Zeroes the padding rows of an expert-sorted buffer (rows r < offsets[E] with token_of[r] ==
 // -1): row_bytes per row, and scale_cols fp32 scales per row when out_scale is given.
