@@ -108,3 +108,44 @@ def test_pipeline_is_deterministic():
         assert torch.equal(getattr(a, name).view(torch.uint8), getattr(b, name).view(torch.uint8)), name
     for name in ("counts", "offsets", "slot_of", "token_of"):
         assert torch.equal(getattr(a.rm, name), getattr(b.rm, name)), name
+
+
+# ---------------------------------------------------------------- randomised sweep
+# TK_FULL_TEST=1 widens it (more seeds and shapes); TK_SEED moves the base seed.
+import os
+
+_FULL = os.environ.get("TK_FULL_TEST", "0") == "1"
+_BASE = int(os.environ.get("TK_SEED", "4242"))
+
+
+@pytest.mark.parametrize("case", range(24 if _FULL else 6))
+def test_random_shapes_against_oracle(case):
+    rng = np.random.default_rng(_BASE + case)
+    E = int(rng.choice([8, 16, 33, 64, 128, 256, 300, 1024]))
+    k = int(rng.integers(1, min(E, 32) + 1))
+    T = int(rng.integers(1, 3000))
+    out_dtype = str(rng.choice(["bf16", "fp8"]))
+    score = str(rng.choice(["softmax", "sigmoid"]))
+    bias = bool(rng.integers(0, 2)) and score == "sigmoid"
+    align = int(rng.choice([1, 1, 4, 128] if E <= 64 else [1, 4]))
+    rmax = T * k + E * (align - 1)
+    hs = [128, 256, 1024, 2176] if out_dtype == "fp8" else [8, 72, 264, 1024, 3000]
+    hs = [h for h in hs if rmax * h <= 40_000_000] or hs[:1]   # keep the CPU-side inputs small
+    H = int(rng.choice(hs))
+    wl = W.Workload(f"rand{case}", T, E, k, H, score, bias, bool(rng.integers(0, 2)), align,
+                    out_dtype, _BASE + 1000 + case)
+    logits, b, x, y = _inputs(wl, "cpu")
+    dev = [t.cuda() if t is not None else None for t in (logits, b, x, y)]
+    run = GpuRun(wl, *dev)
+    assert run.err.item() == 0
+    o_idx, o_w, slot_of, offsets = _check_gate_and_route(wl, run, logits, b)
+    R = int(offsets[-1])
+    if out_dtype == "fp8":
+        q_ref, s_ref = oracle.expand(bf16_bits(x), slot_of, offsets, wl.E, wl.align, oracle.OUT_FP8_E4M3)
+        np.testing.assert_array_equal(run.xq.cpu().numpy()[:R], q_ref[:R])
+        np.testing.assert_array_equal(run.xs.cpu().numpy()[:R], s_ref[:R])
+    else:
+        xe_ref, _ = oracle.expand(bf16_bits(x), slot_of, offsets, wl.E, wl.align)
+        np.testing.assert_array_equal(bf16_bits(run.xe)[:R], xe_ref[:R])
+    out_ref = oracle.reduce(bf16_bits(y), slot_of, o_w)
+    assert bf16_ulp_diff(bf16_bits(run.out), out_ref).max() <= 1
