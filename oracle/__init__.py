@@ -23,7 +23,8 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = LIB if os.path.exists(LIB) else build_oracle()
+        # TKO_LIB points at a planted-mistake build (the mutation test only)
+        path = os.environ.get("TKO_LIB") or (LIB if os.path.exists(LIB) else build_oracle())
         _lib = ctypes.CDLL(path)
         _declare(_lib)
     return _lib

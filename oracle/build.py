@@ -13,6 +13,15 @@ SRC = os.path.join(HERE, "tk_oracle.cpp")
 HDR = os.path.join(HERE, "tk_oracle.h")
 
 
+def build_variant(plant: int, out_path: str) -> str:
+    """Compile the oracle with planted mistake number `plant` (see TKO_PLANT in tk_oracle.cpp)
+    into out_path; used only by the mutation test."""
+    cmd = ["g++", "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+           f"-DTKO_PLANT={int(plant)}", "-o", out_path, SRC]
+    subprocess.run(cmd, check=True)
+    return out_path
+
+
 def build_oracle(force: bool = False) -> str:
     """Compile the oracle if the library is missing or older than its sources; return its path."""
     if not force and os.path.exists(LIB):

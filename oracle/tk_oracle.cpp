@@ -8,6 +8,12 @@
  */
 #include "tk_oracle.h"
 
+/* TKO_PLANT (default 0) compiles one deliberate mistake into the oracle; only the mutation test
+ * (tests/test_oracle_mutations.py) builds such variants, to show that the pins catch each. */
+#ifndef TKO_PLANT
+#define TKO_PLANT 0
+#endif
+
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -59,7 +65,11 @@ float tko_spec_expf(float x) {
     float r = std::fmaf(-n, kLn2Hi, x);
     r = std::fmaf(-n, kLn2Lo, r);
     float p = 0x1.a01a02p-13f;            /* 1/7! */
+#if TKO_PLANT == 1
+    p = std::fmaf(p, r, 0.0f);            /* planted: 1/6! dropped */
+#else
     p = std::fmaf(p, r, 0x1.6c16c2p-10f); /* 1/6! */
+#endif
     p = std::fmaf(p, r, 0x1.111112p-7f);  /* 1/5! */
     p = std::fmaf(p, r, 0x1.555556p-5f);  /* 1/4! */
     p = std::fmaf(p, r, 0x1.555556p-3f);  /* 1/3! */
@@ -107,7 +117,11 @@ uint8_t tko_e4m3_encode(float v) {
     }
     int e = static_cast<int>((float_to_bits(a) >> 23) & 0xFF) - 127; /* floor(log2 a), -6..8 */
     const float quantum = pow2f(e - 3);
+#if TKO_PLANT == 6
+    int m = static_cast<int>(std::round(a / quantum)); /* planted: ties away from zero */
+#else
     int m = static_cast<int>(std::rint(a / quantum)); /* 8..16 */
+#endif
     if (m == 16) { m = 8; e += 1; }
     return static_cast<uint8_t>(sign | ((e + 7) << 3) | (m - 8));
 }
@@ -120,8 +134,12 @@ void tko_e4m3_encode_array(const float* x, uint8_t* y, int64_t n) {
 uint16_t tko_bf16_rne(float f) {
     uint32_t u = float_to_bits(f);
     if ((u & 0x7FFFFFFFu) > 0x7F800000u) return static_cast<uint16_t>((u >> 16) | 0x40u);
+#if TKO_PLANT == 9
+    const uint32_t lsb = 0u; u += 0u * lsb;  /* planted: truncation */
+#else
     const uint32_t lsb = (u >> 16) & 1u;
     u += 0x7FFFu + lsb;
+#endif
     return static_cast<uint16_t>(u >> 16);
 }
 
@@ -160,13 +178,21 @@ int tko_gate_topk(const float* logits, const float* bias, int T, int E, int k, i
             key[e] = kv;
             order[e] = e;
         }
+#if TKO_PLANT == 2
+        std::stable_sort(order.begin(), order.end(),  /* planted: ties to the higher index */
+                         [&](int a, int b) { return key[a] > key[b] || (key[a] == key[b] && a > b); });
+#else
         std::stable_sort(order.begin(), order.end(),
                          [&](int a, int b) { return key[a] > key[b]; });
+#endif
         std::vector<double> s(k);
         if (score_fn == TKO_SCORE_SIGMOID) {
             for (int j = 0; j < k; ++j) {
                 const double lj = static_cast<double>(l[order[j]]);
                 s[j] = 1.0 / (1.0 + std::exp(-lj));
+#if TKO_PLANT == 3
+                if (bias != nullptr) s[j] += bias[order[j]];  /* planted: biased weights */
+#endif
             }
         } else {
             double m = -std::numeric_limits<double>::infinity();
@@ -221,7 +247,11 @@ int tko_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32
     }
     offsets[0] = 0;
     for (int e = 0; e < E; ++e) {
+#if TKO_PLANT == 4
+        const int32_t padded = (counts[e] / align + 1) * align;  /* planted: off-by-one rounding */
+#else
         const int32_t padded = (counts[e] + align - 1) / align * align;
+#endif
         offsets[e + 1] = offsets[e] + padded;
     }
     for (int64_t r = 0; r < rmax; ++r) token_of[r] = -1;
@@ -229,7 +259,11 @@ int tko_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32
     for (int64_t p = 0; p < pairs; ++p) {
         const int e = topk_idx[p];
         if (e < 0 || e >= E) { slot_of[p] = -1; continue; }
+#if TKO_PLANT == 5
+        const int32_t slot = offsets[e] + counts[e] - 1 - fill[e];  /* planted: unstable order */
+#else
         const int32_t slot = offsets[e] + fill[e];
+#endif
         fill[e] += 1;
         slot_of[p] = slot;
         token_of[slot] = static_cast<int32_t>(p / k);
@@ -253,7 +287,11 @@ int tko_quantize_row_e4m3(const uint16_t* xrow, int H, uint8_t* q, float* scales
             for (int c = 0; c < 128; ++c) q[b * 128 + c] = 0x00;
             continue;
         }
+#if TKO_PLANT == 7
+        const float scale = amax / 447.0f;  /* planted: wrong E4M3 maximum */
+#else
         const float scale = amax / 448.0f;
+#endif
         scales[b] = scale;
         for (int c = 0; c < 128; ++c) q[b * 128 + c] = tko_e4m3_encode(bf16_to_float(xrow[b * 128 + c]) / scale);
     }
@@ -311,7 +349,12 @@ int tko_reduce_token(const uint16_t* y, int64_t y_rows, const int32_t* slot_row,
     int bad = 0;
     for (int c = 0; c < H; ++c) {
         float acc = 0.0f;
-        for (int j = 0; j < k; ++j) {
+        for (int jj = 0; jj < k; ++jj) {
+#if TKO_PLANT == 8
+            const int j = k - 1 - jj;  /* planted: reverse slot order */
+#else
+            const int j = jj;
+#endif
             const int64_t slot = slot_row[j];
             if (slot < 0 || slot >= y_rows) { bad = 1; continue; }
             const float wj = w_row != nullptr ? w_row[j] : 1.0f;
@@ -362,7 +405,11 @@ int tko_balance_stats(const float* logits, const int32_t* counts, int T, int E, 
     double acc = 0.0;
     for (int i = 0; i < E; ++i) {
         P[i] = T > 0 ? P[i] / T : 0.0;
+#if TKO_PLANT == 10
+        f[i] = T > 0 ? static_cast<double>(counts[i]) / (static_cast<double>(k) * T) : 0.0;  /* planted */
+#else
         f[i] = T > 0 ? static_cast<double>(E) * counts[i] / (static_cast<double>(k) * T) : 0.0;
+#endif
         acc += f[i] * P[i];
     }
     *loss = acc;
@@ -383,7 +430,11 @@ int tko_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size, int t
     const int lo = tp_rank * el;
     for (int64_t p = 0; p < static_cast<int64_t>(T) * k; ++p) {
         const int e = topk_idx[p];
+#if TKO_PLANT == 12
+        out_idx[p] = (e >= lo && e < lo + el) ? e : -1;  /* planted: not renumbered */
+#else
         out_idx[p] = (e >= lo && e < lo + el) ? e - lo : -1;
+#endif
     }
     return 0;
 }
@@ -420,7 +471,11 @@ int tko_reduce_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_r
                 dot += static_cast<double>(gc) * static_cast<double>(bf16_to_float(y[slot * H + c]));
                 d_y[slot * H + c] = tko_bf16_rne(wj * gc);
             }
+#if TKO_PLANT == 11
+            d_w[p] = static_cast<float>(dot * wj);  /* planted: weighted dot product */
+#else
             d_w[p] = static_cast<float>(dot);
+#endif
         }
     }
     return bad;
