@@ -256,9 +256,19 @@ def run_tk(args, wl):
     from token_routing_gate_b200 import workloads as W
 
     rank, world, local_rank = dist.rank_env()
+    # Test hooks for the multi-rank path on a machine with fewer GPUs than ranks (the kernels of
+    # one rank never wait on another, so ranks may share a GPU): TK_BENCH_DIST_BACKEND=gloo and
+    # TK_BENCH_SAME_DEVICE=1. The numbers of such a run are not a measurement.
+    if os.environ.get("TK_BENCH_SAME_DEVICE") == "1":
+        local_rank = 0
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    dist.init("nccl" if world > 1 else "gloo")
+    backend = os.environ.get("TK_BENCH_DIST_BACKEND", "nccl")
+    dist.init(backend if world > 1 else "gloo")
+    if world > 1 and backend != "nccl":
+        dev_for_collectives = None
+    else:
+        dev_for_collectives = dev
     stream = torch.cuda.current_stream(dev)
 
     swl = wl.with_(seed=dist.shard_seed(wl.seed, rank), param_seed=wl.seed)
@@ -306,7 +316,7 @@ def run_tk(args, wl):
     # Pass 1 (the headline): K steps with nothing between the calls, so each kernel's launch
     # overlaps the end of the previous one as it would in a model.
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier(dev)
+    dist.barrier(dev_for_collectives)
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
         start.record(stream)
@@ -314,18 +324,18 @@ def run_tk(args, wl):
             step()
         end.record(stream)
         torch.cuda.synchronize(dev)
-    dist.barrier(dev)
+    dist.barrier(dev_for_collectives)
     elapsed_s = start.elapsed_time(end) / 1e3
-    max_s = dist.max_over_ranks(elapsed_s, dev)
+    max_s = dist.max_over_ranks(elapsed_s, dev_for_collectives)
     # Pass 2 (the per-kernel breakdown behind the roofline): the same K steps with events
     # between the calls; the events stop one call's launch from overlapping the previous one.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    dist.barrier(dev)
+    dist.barrier(dev_for_collectives)
     torch.cuda.synchronize(dev)
     for i in range(K):
         step(evs[i])
     torch.cuda.synchronize(dev)
-    dist.barrier(dev)
+    dist.barrier(dev_for_collectives)
     names = ["gate", "route_map", "expand", "reduce"]
     k_ms = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K for j, n in enumerate(names)}
     evented_ms = sum(evs[i][0].elapsed_time(evs[i][4]) for i in range(K)) / K
@@ -364,7 +374,7 @@ def run_tk(args, wl):
 
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out,
-                              world)
+                              world, dev_for_collectives)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = time_oracle(wl, args.cpu_seconds)
     if rank == 0:
@@ -373,7 +383,7 @@ def run_tk(args, wl):
     return 0
 
 
-def run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out, world):
+def run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out, world, cdev):
     """Same step through the public calls, with every step's inputs copied in from pinned host
     memory and its result copied back, inside the timed region. Device inputs and outputs are
     double-buffered: step i+1's host-to-device copy and step i-1's device-to-host read run on
@@ -418,7 +428,7 @@ def run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out, 
     for i in range(2):
         e2e_step(i)
     torch.cuda.synchronize(dev)
-    dist.barrier(dev)
+    dist.barrier(cdev)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record(stream)
     s_in.wait_stream(stream)                                  # no copy starts before the clock
@@ -427,8 +437,8 @@ def run_e2e(args, wl, dev, stream, logits, bias, x, y, idx, w, rm, xe, xs, out, 
     stream.wait_stream(s_out)
     e.record(stream)
     torch.cuda.synchronize(dev)
-    dist.barrier(dev)
-    max_s = dist.max_over_ranks(s.elapsed_time(e) / 1e3, dev)
+    dist.barrier(cdev)
+    max_s = dist.max_over_ranks(s.elapsed_time(e) / 1e3, cdev)
     return {"value": dist.aggregate_rate(wl.T * n, world, max_s), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "ms_per_step": 1e3 * max_s / n,
