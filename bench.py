@@ -87,9 +87,15 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def file_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha(kernel_file):
+    """First 16 hex digits of the sha256 of a kernel's .cu file followed by the shared device
+    header it includes (tk_device.cuh): a change to either makes stored counters stale."""
+    csrc = os.path.join(ROOT, "token_routing_gate_b200", "csrc")
+    h = hashlib.sha256()
+    for name in (kernel_file, "tk_device.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel_file, kernel_name, wl_name):
@@ -100,8 +106,7 @@ def ncu_traffic(kernel_file, kernel_name, wl_name):
         with open(path) as f:
             d = json.load(f)
         e = d[wl_name][kernel_name]
-        src = os.path.join(ROOT, "token_routing_gate_b200", "csrc", kernel_file)
-        if e.get("source_sha") != file_sha(src):
+        if e.get("source_sha") != source_sha(kernel_file):
             return None
         return float(e["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError, TypeError):

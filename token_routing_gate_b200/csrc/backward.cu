@@ -30,6 +30,15 @@ constexpr int kChunkBytes = kChunkCh * 2;
 constexpr int kStageBudget = 40 * 1024;
 constexpr int kRegRows = 8;  // up to this k, per-thread register accumulators for d_w
 
+#ifndef TK_BACKWARD_LOAD_POLICY   // L2 policy of the row loads: 0 none, 1 evict-normal, 2 evict-first
+#define TK_BACKWARD_LOAD_POLICY 1
+#endif
+
+__device__ __forceinline__ void load_row(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    if (TK_BACKWARD_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, bar, l2_policy(TK_BACKWARD_LOAD_POLICY));
+    else bulk_load(dst, src, bytes, bar);
+}
+
 struct StageMeta {
     float w[TK_MAX_TOPK];
     int32_t slot[TK_MAX_TOPK];  // -1: skip this row
@@ -115,13 +124,13 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(1 + __popc(vmask)) * bytes);
-                    bulk_load(data + static_cast<size_t>(s) * stage_bytes, g + t * row_bytes + ch0 * 2,
-                              bytes, &full[s]);
+                    load_row(data + static_cast<size_t>(s) * stage_bytes, g + t * row_bytes + ch0 * 2,
+                             bytes, &full[s]);
                 }
                 __syncwarp();
                 if (sl >= 0)
-                    bulk_load(data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(1 + lane) * kChunkBytes,
-                              y + sl * row_bytes + static_cast<int64_t>(ch0) * 2, bytes, &full[s]);
+                    load_row(data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(1 + lane) * kChunkBytes,
+                             y + sl * row_bytes + static_cast<int64_t>(ch0) * 2, bytes, &full[s]);
             }
         }
     } else {

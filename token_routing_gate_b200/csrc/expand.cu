@@ -13,6 +13,9 @@
 //          reduction, scale = amax/448, code = cvt.rn.satfinite.e4m3x2(x/scale) with IEEE
 //          division), writes codes to shared memory, and the elected thread bulk-stores the
 //          code row to the k slots; scales go out as plain stores.
+// The k copies are stored with an L2 evict-first policy: nothing reads them again before they
+// reach DRAM, and without the hint they stay dirty in L2 and are written back while the next
+// kernel runs.
 // Padding rows (only when segments are aligned to more than one row) are zeroed by a separate
 // small kernel that scans token_of for -1 below offsets[E] and bulk-stores zeros over them.
 #include <cuda_runtime.h>
@@ -23,7 +26,25 @@
 namespace tk {
 namespace {
 
+#ifndef TK_EXPAND_STORE_EVICT_FIRST
+#define TK_EXPAND_STORE_EVICT_FIRST 1
+#endif
+
 constexpr uint32_t kCopyChunkBytes = 32768;  // bf16 bytes staged per bulk load
+
+#ifndef TK_EXPAND_LOAD_POLICY   // L2 policy of the token-row loads: 0 none, 1 evict-normal, 2 evict-first
+#define TK_EXPAND_LOAD_POLICY 0
+#endif
+
+__device__ __forceinline__ void load_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    if (TK_EXPAND_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, bar, l2_policy(TK_EXPAND_LOAD_POLICY));
+    else bulk_load(dst, src, bytes, bar);
+}
+
+__device__ __forceinline__ void store_copy(void* dst, const void* src, uint32_t bytes, uint64_t policy) {
+    if (TK_EXPAND_STORE_EVICT_FIRST) bulk_store_hint(dst, src, bytes, policy);
+    else bulk_store(dst, src, bytes);
+}
 constexpr int kFp8Threads = 256;
 constexpr int kFp8ChunkChannels = 8192;      // channels quantised per stage
 
@@ -51,6 +72,7 @@ expand_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ sl
     }
     const uint8_t* src = x + t * row_bytes;
     const uint32_t nchunks = (row_bytes + kCopyChunkBytes - 1) / kCopyChunkBytes;
+    const uint64_t policy = l2_policy_evict_first();
     for (uint32_t c = 0; c < nchunks; ++c) {
         const uint32_t off = c * kCopyChunkBytes;
         const uint32_t bytes = min(kCopyChunkBytes, row_bytes - off);
@@ -61,7 +83,7 @@ expand_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ sl
                 fence_proxy_async_smem();
             }
             mbar_arrive_expect_tx(&bar, bytes);
-            bulk_load(stage, src + off, bytes, &bar);
+            load_copy(stage, src + off, bytes, &bar);
             ok = mbar_wait_bounded(&bar, c & 1u) ? 1 : 0;
             if (!ok) {
                 flag_error(err_flag, TK_DEVERR_TIMEOUT);
@@ -72,7 +94,7 @@ expand_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ sl
         if (!ok) break;
         for (int j = 0; j < k; ++j) {
             const int64_t s = __shfl_sync(kFullMask, my_slot, j);
-            if (lane == 0 && s >= 0) bulk_store(out + s * row_bytes + off, stage, bytes);
+            if (lane == 0 && s >= 0) store_copy(out + s * row_bytes + off, stage, bytes, policy);
         }
         if (lane == 0) bulk_commit();
     }
@@ -110,6 +132,7 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
     }
     const int nb_row = H / 128;
     const int nchunks = (H + chunk - 1) / chunk;
+    const uint64_t policy = l2_policy_evict_first();
     for (int c = 0; c < nchunks; ++c) {
         const int ch0 = c * chunk;
         const int chn = min(chunk, H - ch0);
@@ -117,7 +140,7 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
             if (c > 0) bulk_wait_read_all();
             fence_proxy_async_smem();
             mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(chn) * 2u);
-            bulk_load(xin, x + t * H + ch0, static_cast<uint32_t>(chn) * 2u, &bar);
+            load_copy(xin, x + t * H + ch0, static_cast<uint32_t>(chn) * 2u, &bar);
             int ok = mbar_wait_bounded(&bar, static_cast<uint32_t>(c) & 1u) ? 1 : 0;
             if (!ok) {
                 flag_error(err_flag, TK_DEVERR_TIMEOUT);
@@ -154,7 +177,7 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
         if (tid == 0) {
             for (int j = 0; j < k; ++j) {
                 const int64_t s = slots[j];
-                if (s >= 0) bulk_store(out_q + s * H + ch0, qo, static_cast<uint32_t>(chn));
+                if (s >= 0) store_copy(out_q + s * H + ch0, qo, static_cast<uint32_t>(chn), policy);
             }
             bulk_commit();
         }

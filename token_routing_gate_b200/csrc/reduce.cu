@@ -15,8 +15,12 @@
 // The ring has S stages with S*k*2 KB <= 32 KB (two at k = 8), so an SM holds about six CTAs and
 // up to ~190 KB of loads in flight. A measured sweep on B200 (ring depth, chunk width, consumer
 // warps) put this shape at the HBM copy roofline; deeper rings with fewer CTAs per SM were up to
-// 30% slower. The grid is persistent (SM count x CTAs per SM) and CTAs stride over units. Every wait is bounded (1 s); a timeout flags TK_DEVERR_TIMEOUT and ends the
-// CTA's loop.
+// 30% slower. The grid is persistent (SM count x CTAs per SM) and CTAs stride over units.
+// The row loads carry an explicit L2 evict-normal policy. Measured on B200 at T=8192, H=7168,
+// k=8: with it the reduce after dispatch and the reduce run back to back were both faster than
+// with no policy operand (forward step 366.8 -> 364.9 us; back-to-back reduce 155.5 -> 152.9 us).
+// Evict-first won the forward step (361.7 us) but cost 16 us back to back, so it is not used.
+// Every wait is bounded (1 s); a timeout flags TK_DEVERR_TIMEOUT and ends the CTA's loop.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -31,6 +35,9 @@ namespace {
 #endif
 #ifndef TK_REDUCE_VECS_PER_THREAD
 #define TK_REDUCE_VECS_PER_THREAD 1
+#endif
+#ifndef TK_REDUCE_LOAD_POLICY   // L2 policy of the row loads: 0 none, 1 evict-normal, 2 evict-first
+#define TK_REDUCE_LOAD_POLICY 1
 #endif
 #ifndef TK_REDUCE_STAGE_KB
 #define TK_REDUCE_STAGE_KB 32
@@ -145,9 +152,12 @@ reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __re
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(vmask)) * bytes);
             __syncwarp();
-            if (sl >= 0)
-                bulk_load(data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * kChunkBytes,
-                          y + sl * row_bytes + static_cast<int64_t>(ch0) * 2, bytes, &full[s]);
+            if (sl >= 0) {
+                uint8_t* dst = data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * kChunkBytes;
+                const uint8_t* src = y + sl * row_bytes + static_cast<int64_t>(ch0) * 2;
+                if (TK_REDUCE_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, &full[s], l2_policy(TK_REDUCE_LOAD_POLICY));
+                else bulk_load(dst, src, bytes, &full[s]);
+            }
         }
     } else {
         // ---------------- consumers
