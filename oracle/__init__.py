@@ -68,6 +68,15 @@ def _declare(L):
     L.tko_tp_mask.restype = i32
     L.tko_reduce_backward.argtypes = [vp, vp, i64, vp, vp, vp, i32, i32, i32, i32, vp, vp]
     L.tko_reduce_backward.restype = i32
+    L.tko_ep_layout.argtypes = [vp, i32, i32, i32, i32, vp, vp]
+    L.tko_ep_layout.restype = i32
+    L.tko_ep_recv_bases.argtypes = [vp, i32, vp, vp]
+    L.tko_ep_recv_bases.restype = i32
+    L.tko_ep_dispatch.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i32, vp, vp,
+                                  vp, vp]
+    L.tko_ep_dispatch.restype = i32
+    L.tko_ep_combine.argtypes = [vp, vp, vp, i32, i32, i32, vp]
+    L.tko_ep_combine.restype = i32
 
 
 def _c(a, dtype):
@@ -222,3 +231,95 @@ def reduce_backward(grad_bits, y_bits, slot_of, offsets, w, E):
     if rc < 0:
         raise ValueError("tko_reduce_backward rejected its arguments")
     return d_y, d_w, rc
+
+
+# ---------------------------------------------------------------- expert-parallel dispatch / combine
+def ep_layout(topk_idx, E, G):
+    """(send_counts [G], dest_pos [T, G]) of one source rank."""
+    topk_idx = _c(topk_idx, np.int32)
+    T, k = topk_idx.shape
+    counts = np.empty(G, dtype=np.int32)
+    dest_pos = np.empty((T, G), dtype=np.int32)
+    rc = lib().tko_ep_layout(_p(topk_idx), T, E, k, G, _p(counts), _p(dest_pos))
+    if rc < 0:
+        raise ValueError(f"tko_ep_layout rejected its arguments (rc={rc})")
+    return counts, dest_pos
+
+
+def ep_recv_bases(count_matrix):
+    """count_matrix [G, G] (source, destination) -> (base [G, G] int64, recv_rows [G] int64)."""
+    cm = _c(count_matrix, np.int32)
+    G = cm.shape[0]
+    base = np.empty((G, G), dtype=np.int64)
+    recv = np.empty(G, dtype=np.int64)
+    if lib().tko_ep_recv_bases(_p(cm), G, _p(base), _p(recv)) < 0:
+        raise ValueError("tko_ep_recv_bases rejected its arguments")
+    return base, recv
+
+
+def ep_dispatch(x_bits, topk_idx, topk_w, dest_pos, E, G, d, base_row, recv, out_dtype=OUT_BF16):
+    """Writes one source's rows bound for rank d into recv = (recv_x, recv_scale, recv_idx,
+    recv_w), the destination's receive buffers (numpy arrays, modified in place)."""
+    x_bits = _c(x_bits, np.uint16)
+    topk_idx = _c(topk_idx, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    dest_pos = _c(dest_pos, np.int32)
+    T, H = x_bits.shape
+    k = topk_idx.shape[1]
+    rx, rs, ri, rw = recv
+    rc = lib().tko_ep_dispatch(_p(x_bits), _p(topk_idx), _p(topk_w), _p(dest_pos), T, E, k, H, G,
+                               d, int(base_row), out_dtype, _p(rx), _p(rs), _p(ri), _p(rw))
+    if rc < 0:
+        raise ValueError(f"tko_ep_dispatch rejected its arguments (rc={rc})")
+
+
+def ep_combine(partials, base_rows, dest_pos):
+    """partials[d]: bf16 bits [rows_d, H] of every rank d; base_rows [G]: this source's first row
+    in each rank's buffer; dest_pos [T, G] of this source. Returns out bits [T, H]."""
+    dest_pos = _c(dest_pos, np.int32)
+    T, G = dest_pos.shape
+    parts = [_c(a, np.uint16) for a in partials]
+    H = parts[0].shape[1]
+    ptrs = (ctypes.c_void_p * G)(*[a.ctypes.data for a in parts])
+    base = _c(base_rows, np.int64)
+    out = np.empty((T, H), dtype=np.uint16)
+    if lib().tko_ep_combine(ptrs, _p(base), _p(dest_pos), T, G, H, _p(out)) < 0:
+        raise ValueError("tko_ep_combine rejected its arguments")
+    return out
+
+
+def ep_forward(xs, idxs, ws, make_y, E, G, align=1, out_dtype=OUT_BF16):
+    """The whole expert-parallel forward over G ranks, stated step by step with the functions
+    above (and the single-rank route map and reduce on each destination). xs[s], idxs[s],
+    ws[s]: source rank s's token rows (bf16 bits), choices and weights. make_y(d, rows) returns
+    rank d's expert outputs (bf16 bits [rows, H]) indexed by its local slots. Returns a dict of
+    every intermediate and the per-source outputs."""
+    k = idxs[0].shape[1]
+    H = xs[0].shape[1]
+    el = E // G
+    lay = [ep_layout(idxs[s], E, G) for s in range(G)]
+    cm = np.stack([c for c, _ in lay])
+    base, recv_rows = ep_recv_bases(cm)
+    recv = []
+    for d in range(G):
+        n = int(recv_rows[d])
+        if out_dtype == OUT_BF16:
+            rx, rs = np.zeros((n, H), dtype=np.uint16), np.zeros((n, 1), dtype=np.float32)
+        else:
+            rx, rs = np.zeros((n, H), dtype=np.uint8), np.zeros((n, H // 128), dtype=np.float32)
+        buf = (rx, rs, np.full((n, k), -7, dtype=np.int32), np.zeros((n, k), dtype=np.float32))
+        for s in range(G):
+            ep_dispatch(xs[s], idxs[s], ws[s], lay[s][1], E, G, d, base[s, d], buf, out_dtype)
+        recv.append(buf)
+    dest, partials = [], []
+    for d in range(G):
+        n = int(recv_rows[d])
+        counts, offsets, slot_of, token_of, rc = route_map(recv[d][2], el, align)
+        y = make_y(d, max(max_rows(n, el, k, align), 1))
+        part = reduce(y, slot_of, recv[d][3]) if n > 0 else np.zeros((0, H), dtype=np.uint16)
+        dest.append({"counts": counts, "offsets": offsets, "slot_of": slot_of, "token_of": token_of,
+                     "y": y})
+        partials.append(part if n > 0 else np.zeros((1, H), dtype=np.uint16))
+    outs = [ep_combine(partials, base[s], lay[s][1]) for s in range(G)]
+    return {"layout": lay, "count_matrix": cm, "base": base, "recv_rows": recv_rows, "recv": recv,
+            "dest": dest, "partials": partials, "out": outs}

@@ -481,4 +481,118 @@ int tko_reduce_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_r
     return bad;
 }
 
+/* ------------------------------------------------------------------------------------------
+ * Expert-parallel dispatch and combine over G ranks. Sources: 147227.xyz "刚刚！DeepSeek开源高
+ * 性能GPU算子库TileKernels" (its DeepEP paragraph: an expert-parallel all-to-all library over
+ * NVLink with native FP8 dispatch) and 機器之心 "剛剛，DeepSeek開始頻繁更新：Tile Kernels、
+ * DeepEP V2", section "性能表現" (the DeepSeek-V3 setting with FP8 dispatch and BF16 combine).
+ * Neither page gives a layout or a formula; the readings, each the plainest one:
+ *  - experts are owned in G contiguous groups of E/G (expert e lives on rank e / (E/G));
+ *  - a token goes once to every rank that owns at least one of its experts (not once per
+ *    expert); masked pairs (expert -1) go nowhere;
+ *  - a destination's receive buffer holds the rows of source 0, then source 1, ..., each
+ *    source's rows in token order;
+ *  - each received row carries the token's k choices renumbered to the destination's local
+ *    experts (-1 for experts of other ranks) and the matching weights (0 for those);
+ *  - the destination combines its own experts' rows of a received token like the single-GPU
+ *    reduce (fp32 fmaf in slot order) and rounds the partial sum to bf16 (BF16 combine);
+ *  - the source adds the bf16 partial rows of the token's destinations in ascending rank
+ *    order in fp32 and rounds once to bf16.
+ * ---------------------------------------------------------------------------------------- */
+static int ep_owner(int e, int E, int G) {
+#if TKO_PLANT == 14
+    return e % G;  /* planted: experts dealt round-robin over the ranks */
+#else
+    return e / (E / G);
+#endif
+}
+
+int tko_ep_layout(const int32_t* topk_idx, int T, int E, int k, int G, int32_t* send_counts,
+                  int32_t* dest_pos) {
+    if (T < 0 || E < 1 || k < 1 || G < 1 || E % G != 0) return -1;
+    for (int d = 0; d < G; ++d) send_counts[d] = 0;
+    std::vector<char> goes(G);
+    for (int t = 0; t < T; ++t) {
+        std::fill(goes.begin(), goes.end(), 0);
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[static_cast<int64_t>(t) * k + j];
+            if (e == -1) continue;
+            if (e < 0 || e >= E) return -2;
+            goes[ep_owner(e, E, G)] = 1;
+        }
+        for (int d = 0; d < G; ++d)
+            dest_pos[static_cast<int64_t>(t) * G + d] = goes[d] ? send_counts[d]++ : -1;
+    }
+    return 0;
+}
+
+int tko_ep_recv_bases(const int32_t* count_matrix, int G, int64_t* base, int64_t* recv_rows) {
+    if (G < 1) return -1;
+    for (int d = 0; d < G; ++d) {
+        int64_t acc = 0;
+        for (int s = 0; s < G; ++s) {
+            base[static_cast<int64_t>(s) * G + d] = acc;
+            acc += count_matrix[static_cast<int64_t>(s) * G + d];
+        }
+        recv_rows[d] = acc;
+    }
+    return 0;
+}
+
+int tko_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
+                    const int32_t* dest_pos, int T, int E, int k, int H, int G, int d,
+                    int64_t base_row, int out_dtype, void* recv_x, float* recv_scale,
+                    int32_t* recv_idx, float* recv_w) {
+    if (T < 0 || E < 1 || k < 1 || H <= 0 || G < 1 || E % G != 0 || d < 0 || d >= G) return -1;
+    if (out_dtype != TKO_OUT_BF16 && out_dtype != TKO_OUT_FP8_E4M3) return -1;
+    if (out_dtype == TKO_OUT_FP8_E4M3 && H % 128 != 0) return -1;
+    const int el = E / G;
+    for (int t = 0; t < T; ++t) {
+        const int pos = dest_pos[static_cast<int64_t>(t) * G + d];
+        if (pos < 0) continue;
+        const int64_t row = base_row + pos;
+        const uint16_t* xr = x + static_cast<int64_t>(t) * H;
+        if (out_dtype == TKO_OUT_BF16) {
+            std::memcpy(static_cast<uint16_t*>(recv_x) + row * H, xr, sizeof(uint16_t) * H);
+        } else {
+            tko_quantize_row_e4m3(xr, H, static_cast<uint8_t*>(recv_x) + row * H,
+                                  recv_scale + row * (H / 128));
+        }
+        for (int j = 0; j < k; ++j) {
+            const int64_t p = static_cast<int64_t>(t) * k + j;
+            const int e = topk_idx[p];
+            const bool mine = e >= 0 && e < E && ep_owner(e, E, G) == d;
+#if TKO_PLANT == 15
+            recv_idx[row * k + j] = mine ? e : -1;  /* planted: global expert id sent */
+#else
+            recv_idx[row * k + j] = mine ? e - d * el : -1;
+#endif
+            recv_w[row * k + j] = mine ? topk_w[p] : 0.0f;
+        }
+    }
+    return 0;
+}
+
+int tko_ep_combine(const uint16_t* const* partial, const int64_t* base_row,
+                   const int32_t* dest_pos, int T, int G, int H, uint16_t* out) {
+    if (T < 0 || G < 1 || H <= 0) return -1;
+    for (int t = 0; t < T; ++t) {
+        for (int c = 0; c < H; ++c) {
+            float acc = 0.0f;
+            for (int dd = 0; dd < G; ++dd) {
+#if TKO_PLANT == 13
+                const int d = G - 1 - dd;  /* planted: descending rank order */
+#else
+                const int d = dd;
+#endif
+                const int pos = dest_pos[static_cast<int64_t>(t) * G + d];
+                if (pos < 0) continue;
+                acc = acc + bf16_to_float(partial[d][(base_row[d] + pos) * H + c]);
+            }
+            out[static_cast<int64_t>(t) * H + c] = tko_bf16_rne(acc);
+        }
+    }
+    return 0;
+}
+
 }  // extern "C"

@@ -118,6 +118,29 @@ int tko_reduce_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_r
                         const int32_t* slot_of, const int32_t* offsets, const float* w, int T,
                         int E, int k, int H, uint16_t* d_y, float* d_w);
 
+/* ---- expert-parallel dispatch / combine over G ranks (experts in G contiguous groups) ---- */
+
+/* For one source rank: dest_pos[t*G+d] = position of token t among this rank's tokens that go
+ * to rank d (token order), or -1 when no expert of t lives on d; send_counts[d] = how many go.
+ * Returns -2 for an expert outside [0,E) other than the masked -1. */
+int tko_ep_layout(const int32_t* topk_idx, int T, int E, int k, int G, int32_t* send_counts,
+                  int32_t* dest_pos);
+/* From the G x G matrix count_matrix[s*G+d] (rows source s sends to rank d):
+ * base[s*G+d] = first row of source s in rank d's receive buffer (sources in rank order),
+ * recv_rows[d] = rows rank d receives. */
+int tko_ep_recv_bases(const int32_t* count_matrix, int G, int64_t* base, int64_t* recv_rows);
+/* Writes source rank's tokens bound for rank d into d's receive buffer at rows
+ * base_row + dest_pos[t*G+d]: the row (bf16, or E4M3 codes + per-128-channel scales), the k
+ * choices renumbered to d's local experts (-1 elsewhere) and their weights (0 elsewhere). */
+int tko_ep_dispatch(const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
+                    const int32_t* dest_pos, int T, int E, int k, int H, int G, int d,
+                    int64_t base_row, int out_dtype, void* recv_x, float* recv_scale,
+                    int32_t* recv_idx, float* recv_w);
+/* out[t] = bf16( sum over d ascending with dest_pos[t*G+d] >= 0 of
+ *                fp32(partial[d][base_row[d] + dest_pos[t*G+d]]) ), fp32 adds. */
+int tko_ep_combine(const uint16_t* const* partial, const int64_t* base_row,
+                   const int32_t* dest_pos, int T, int G, int H, uint16_t* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,7 +1,8 @@
 """Mutation test of the oracle's pins: each planted mistake (a dropped series term, the wrong
 tie-break, biased weights, an off-by-one padding, unstable slots, the wrong E4M3 rounding or
 scale, the wrong reduction order, truncating bf16 rounding, a missing factor in the balance
-loss, a weighted gradient, an un-renumbered TP mask) is compiled into a copy of the oracle,
+loss, a weighted gradient, an un-renumbered TP mask, the expert-parallel combine in the wrong
+rank order, experts dealt round-robin over ranks, global expert ids sent) is compiled into a copy of the oracle,
 and the pins that cover that step must fail against it. The unplanted build must pass them."""
 import os
 import subprocess
@@ -26,6 +27,9 @@ MUTATIONS = {
     10: "balance_stats",
     11: "reduce_backward",
     12: "tp_mask",
+    13: "ep_combine_rank_order",
+    14: "ep_layout or ep_dispatch",
+    15: "ep_dispatch",
 }
 
 

@@ -533,3 +533,146 @@ def test_reduce_backward_unit_weights_and_padding(oracle_lib):
     # and the fp32/bf16 reduce of G is that sum rounded (within the reduce's own bound)
     exact = Gf[slot_of].sum(1)
     assert np.all(np.abs(_bits_to_f32(back) - exact) <= k * 2.0 ** -24 * np.abs(Gf[slot_of]).sum(1) + np.abs(exact) * 2.0 ** -8)
+
+
+# ---------------------------------------------------------------- expert-parallel dispatch / combine
+def _ep_choices(rng, T, E, k, masked=0.0):
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    if masked:
+        idx[rng.random(idx.shape) < masked] = -1
+    return idx
+
+
+def _bf16_bits(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_ep_layout_invariants(oracle_lib):
+    # dest_pos >= 0 exactly for the ranks owning one of the token's experts (E/G contiguous
+    # experts per rank), numbered 0, 1, 2, ... in token order; counts are the totals.
+    rng = np.random.default_rng(31)
+    for G, E, k, T in [(1, 8, 3, 20), (2, 8, 3, 50), (4, 16, 5, 64), (8, 64, 8, 40), (3, 12, 12, 9)]:
+        idx = _ep_choices(rng, T, E, k, masked=0.2)
+        counts, dest = oracle_lib.ep_layout(idx, E, G)
+        group = E // G
+        for d in range(G):
+            goes = np.array([any(e >= 0 and e // group == d for e in row) for row in idx])
+            assert np.array_equal(dest[:, d] >= 0, goes)
+            assert dest[goes, d].tolist() == list(range(int(goes.sum())))
+            assert counts[d] == goes.sum()
+
+
+def test_ep_layout_masked_and_bad_index(oracle_lib):
+    idx = np.array([[-1, -1], [3, -1]], dtype=np.int32)
+    counts, dest = oracle_lib.ep_layout(idx, 4, 2)
+    assert dest.tolist() == [[-1, -1], [-1, 0]] and counts.tolist() == [0, 1]
+    with pytest.raises(ValueError):
+        oracle_lib.ep_layout(np.array([[4, 0]], dtype=np.int32), 4, 2)
+    with pytest.raises(ValueError):
+        oracle_lib.ep_layout(idx, 6, 4)   # E not a multiple of G
+
+
+def test_ep_recv_bases_hand_case(oracle_lib):
+    # rank d receives source 0's rows first, then source 1's, ...: base[s][d] = sum_{s'<s} c[s'][d]
+    base, recv = oracle_lib.ep_recv_bases(np.array([[1, 2, 0], [3, 4, 5], [0, 6, 7]]))
+    assert base.tolist() == [[0, 0, 0], [1, 2, 0], [4, 6, 5]]
+    assert recv.tolist() == [4, 12, 12]
+
+
+@pytest.mark.parametrize("out_dtype", [0, 1], ids=["bf16", "fp8"])
+def test_ep_dispatch_rows_and_local_ids(oracle_lib, out_dtype):
+    rng = np.random.default_rng(33)
+    G, E, k, T, H = 4, 16, 3, 30, 256
+    group = E // G
+    xs = [_bf16_bits(rng.standard_normal((T, H))) for _ in range(G)]
+    idxs = [_ep_choices(rng, T, E, k, masked=0.1) for _ in range(G)]
+    ws = [rng.random((T, k)).astype(np.float32) for _ in range(G)]
+    r = oracle_lib.ep_forward(xs, idxs, ws, lambda d, n: np.zeros((n, H), np.uint16), E, G,
+                              out_dtype=out_dtype)
+    for d in range(G):
+        rx, rs, ri, rw = r["recv"][d]
+        row = 0
+        for s in range(G):
+            dest = r["layout"][s][1]
+            for t in range(T):
+                if dest[t, d] < 0:
+                    continue
+                if out_dtype == 0:
+                    np.testing.assert_array_equal(rx[row], xs[s][t])
+                else:
+                    q, sc = oracle_lib.quantize_row_e4m3(xs[s][t])
+                    np.testing.assert_array_equal(rx[row], q)
+                    np.testing.assert_array_equal(rs[row], sc)
+                for j in range(k):
+                    e = idxs[s][t, j]
+                    mine = e >= 0 and e // group == d
+                    assert ri[row, j] == (e - d * group if mine else -1)
+                    assert rw[row, j] == (ws[s][t, j] if mine else 0.0)
+                row += 1
+        assert row == r["recv_rows"][d]
+
+
+def test_ep_combine_rank_order(oracle_lib):
+    # fp32 adds in ascending rank order: 2^27 + (-2^27) + 1 = 1; the reverse order gives 0
+    H = 8
+    parts = [_bf16_bits(np.full((1, H), v)) for v in (2.0 ** 27, -(2.0 ** 27), 1.0)]
+    out = oracle_lib.ep_combine(parts, np.zeros(3, np.int64), np.zeros((1, 3), np.int32))
+    assert np.all(out == _bf16_bits(np.ones((1, H))))
+    # a token no rank received combines to zero
+    out = oracle_lib.ep_combine(parts, np.zeros(3, np.int64), np.full((1, 3), -1, np.int32))
+    assert np.all(out == 0)
+
+
+def test_ep_one_rank_is_the_single_rank_path(oracle_lib):
+    rng = np.random.default_rng(35)
+    E, k, T, H = 12, 4, 40, 64
+    x = _bf16_bits(rng.standard_normal((T, H)))
+    idx = _ep_choices(rng, T, E, k)
+    w = rng.random((T, k)).astype(np.float32)
+    ys = {}
+
+    def make_y(d, n):
+        ys[d] = _bf16_bits(rng.standard_normal((n, H)))
+        return ys[d]
+
+    r = oracle_lib.ep_forward([x], [idx], [w], make_y, E, 1)
+    np.testing.assert_array_equal(r["recv"][0][0], x)
+    counts, offsets, slot_of, token_of, _ = oracle_lib.route_map(idx, E, 1)
+    np.testing.assert_array_equal(r["out"][0], oracle_lib.reduce(ys[0], slot_of, w))
+
+
+def test_ep_tokens_on_one_rank_match_that_ranks_reduce(oracle_lib):
+    rng = np.random.default_rng(36)
+    G, E, k, T, H = 4, 32, 4, 25, 40
+    group = E // G
+    idxs = []
+    for _ in range(G):
+        home = rng.integers(0, G, T)
+        idxs.append(np.stack([home[t] * group + rng.choice(group, k, replace=False)
+                              for t in range(T)]).astype(np.int32))
+    xs = [_bf16_bits(rng.standard_normal((T, H))) for _ in range(G)]
+    ws = [rng.random((T, k)).astype(np.float32) for _ in range(G)]
+    r = oracle_lib.ep_forward(xs, idxs, ws, lambda d, n: _bf16_bits(rng.standard_normal((n, H))),
+                              E, G)
+    for s in range(G):
+        dest = r["layout"][s][1]
+        for t in range(T):
+            (d,) = np.nonzero(dest[t] >= 0)[0]
+            row = r["base"][s, d] + dest[t, d]
+            D = r["dest"][d]
+            want = oracle_lib.reduce_token(D["y"], D["slot_of"][row], ws[s][t])
+            np.testing.assert_array_equal(r["out"][s][t], want)
+
+
+def test_ep_closed_form_equal_rows(oracle_lib):
+    # every expert output row is v and every weight 1/4: rank d's partial is (n_d/4) v exactly,
+    # and the partials of a token add up to v exactly, whatever the split over ranks
+    rng = np.random.default_rng(37)
+    G, E, k, T, H = 4, 16, 4, 30, 16
+    v = _bf16_bits(rng.integers(-64, 64, H) / 8.0)
+    xs = [_bf16_bits(rng.standard_normal((T, H))) for _ in range(G)]
+    idxs = [_ep_choices(rng, T, E, k) for _ in range(G)]
+    ws = [np.full((T, k), 0.25, np.float32) for _ in range(G)]
+    r = oracle_lib.ep_forward(xs, idxs, ws, lambda d, n: np.tile(v, (n, 1)), E, G)
+    for s in range(G):
+        assert np.all(r["out"][s] == v[None, :])
