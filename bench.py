@@ -42,9 +42,14 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for cpu_baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--op", choices=["step", "backward", "stats"], default="step",
+    p.add_argument("--op", choices=["step", "backward", "stats", "ep"], default="step",
                    help="step: the forward path (the benchmark's headline); backward: reduce and "
-                        "expand backward; stats: load-balance statistics and the TP mask")
+                        "expand backward; stats: load-balance statistics and the TP mask; ep: "
+                        "expert-parallel dispatch/combine of the batch over --ep-ranks ranks run "
+                        "on one GPU")
+    p.add_argument("--ep-ranks", type=int, default=8, help="ranks of the --op ep run")
+    p.add_argument("--ep-dtype", choices=["bf16", "fp8"], default="fp8",
+                   help="dispatch format of the --op ep run (the pages' setting: FP8 dispatch)")
     return p.parse_args()
 
 
@@ -516,6 +521,80 @@ def run_op(args, wl):
     return 0
 
 
+def run_ep(args, wl):
+    """Expert-parallel dispatch -> experts' combine -> combine of the workload's batch split over
+    G ranks, all run on one GPU (VirtualRanks). The "transfers" are writes and reads of this
+    GPU's own memory, so the numbers are HBM numbers of the EP kernels, not NVLink numbers."""
+    import torch
+    from token_routing_gate_b200 import ep, tk
+    from token_routing_gate_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    G = args.ep_ranks
+    T, E, k, H = wl.T, wl.E, wl.k, wl.H
+    if T % G or E % G:
+        raise SystemExit(f"--ep-ranks {G} must divide T={T} and E={E}")
+    Tr = T // G
+    logits, bias = W.gate_inputs(wl, dev)
+    x = W.activations(wl, dev)
+    idx, w = tk.gate_topk(logits, k, wl.score, bias)
+    xs = [x[s * Tr:(s + 1) * Tr] for s in range(G)]
+    idxs = [idx[s * Tr:(s + 1) * Tr].contiguous() for s in range(G)]
+    ws = [w[s * Tr:(s + 1) * Tr].contiguous() for s in range(G)]
+    vr = ep.VirtualRanks(G, E, k, H, Tr, args.ep_dtype, 1, dev)
+    y = W.expert_outputs(wl, dev, rows=tk.max_rows(T, E // G, k, 1))   # shared by the ranks
+    outs = [torch.empty(Tr, H, dtype=torch.bfloat16, device=dev) for _ in range(G)]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def expert_fn(d, bufs, n, rm):
+        return y
+
+    names = ["layout", "dispatch", "experts", "combine"]
+
+    def step(evs=None):
+        if evs is None:
+            return vr.step(xs, idxs, ws, expert_fn, outs, err, stream)
+        evs["start"].record(stream)
+        return vr.step(xs, idxs, ws, expert_fn, outs, err, stream, mark=lambda n: evs[n].record(stream))
+
+    for _ in range(args.warmup):
+        res = step()
+    torch.cuda.synchronize(dev)
+    if err.item() != 0:
+        raise SystemExit(f"device error flag {err.item()}")
+    recv = res["recv_rows"]
+    K = args.steps
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in ["start"] + names} for _ in range(K)]
+    with ClockSampler(dev.index) as clocks:
+        for i in range(K):
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    prev = ["start"] + names[:-1]
+    phase_us = {n: 1e3 * sum(e[p].elapsed_time(e[n]) for e in evs) / K for p, n in zip(prev, names)}
+    step_ms = sum(e["start"].elapsed_time(e["combine"]) for e in evs) / K
+    sent_rows = int(recv.sum())
+    row_out = H if args.ep_dtype == "fp8" else 2 * H
+    scale_b = 4 * (H // 128) if args.ep_dtype == "fp8" else 0
+    disp_bytes = T * 2 * H + sent_rows * (row_out + scale_b + 8 * k) + T * k * 8
+    comb_bytes = sent_rows * 2 * H + T * 2 * H
+    line = {"metric": f"expert-parallel dispatch + combine tokens/s, {G} ranks on one GPU",
+            "op": "ep", "value": T / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "dtype": args.ep_dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "T": T, "E": E, "k": k, "H": H, "ranks": G,
+                       "tokens_per_rank": Tr, "rows_sent": sent_rows,
+                       "emulated": "all ranks on one GPU: transfers are local HBM traffic"},
+            "phases_us": phase_us,
+            "hbm_gbs": {"dispatch": disp_bytes / (phase_us["dispatch"] * 1e3),
+                        "combine": comb_bytes / (phase_us["combine"] * 1e3)},
+            "bytes": {"dispatch": disp_bytes, "combine": comb_bytes},
+            "clocks": clocks.summary(), "gpu_launches": None}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     from token_routing_gate_b200 import workloads as W
@@ -524,6 +603,8 @@ def main():
         wl = wl.with_(T=args.tokens, name=f"{wl.name}_T{args.tokens}")
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.op == "ep":
+        return run_ep(args, wl)
     if args.op != "step":
         return run_op(args, wl)
     return run_tk(args, wl)

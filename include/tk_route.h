@@ -63,6 +63,7 @@ typedef enum tk_out_dtype { TK_OUT_BF16 = 0, TK_OUT_FP8_E4M3 = 1 } tk_out_dtype;
 /* Limits of the warp-per-token gate. */
 #define TK_MAX_EXPERTS 1024
 #define TK_MAX_TOPK 32
+#define TK_MAX_EP_RANKS 32   /* expert-parallel ranks (tk_ep_*) */
 
 /*
  * Gate: expert scoring, top-k selection and weight normalisation (機器之心 "Tile Kernels"
@@ -96,7 +97,9 @@ TK_API size_t tk_route_map_workspace_bytes(int T, int E, int k);
 /*
  * Token-to-expert map (機器之心 "Tile Kernels" feature list: token-to-expert mapping).
  * Pair p = t*k + j.
- *   topk_idx  device, int32 [T, k] (k distinct experts per token)
+ *   topk_idx  device, int32 [T, k], 1 <= k <= 32: a token's experts other than -1 are
+ *             distinct (so k may exceed E when pairs are masked, as after tk_tp_mask or on an
+ *             expert-parallel destination)
  *   align     >= 1 (<= 4096): each expert's segment is padded to a multiple of align rows
  *   counts    device, int32 [E]: pairs routed to each expert
  *   offsets   device, int32 [E+1]: offsets[0] = 0, offsets[e+1] = offsets[e] +
@@ -224,6 +227,93 @@ TK_API tk_status tk_reduce_backward(const void* grad_out, const void* y, int64_t
 TK_API tk_status tk_expand_backward(const void* d_xe, int64_t xe_rows, const int32_t* slot_of,
                                     int T, int k, int H, void* d_x, int32_t* err_flag,
                                     void* stream);
+
+/*
+ * Expert-parallel dispatch and combine over G ranks (147227.xyz "刚刚！DeepSeek开源高性能GPU算子库
+ * TileKernels", its DeepEP paragraph: an expert-parallel all-to-all over NVLink with native FP8
+ * dispatch; 機器之心 "剛剛，DeepSeek開始頻繁更新：Tile Kernels、DeepEP V2", section "性能表現":
+ * FP8 dispatch, BF16 combine). Neither page gives a layout; the one used here:
+ *   - expert e lives on rank e / (E/G) (G contiguous groups; G must divide E);
+ *   - a token goes once to each rank that owns at least one of its experts;
+ *   - rank d's receive buffers hold the rows of source rank 0, then 1, ..., each source's rows
+ *     in token order (a source's first row there is its base_row, the sum of the rows lower
+ *     ranks send to d -- the caller exchanges the G x G send counts to get it);
+ *   - each received row carries the token's k choices renumbered to d's local experts
+ *     (0 .. E/G-1; -1 for other ranks' experts) and the weights (0 for other ranks' experts),
+ *     so rank d routes them with tk_route_map (E/G experts), expands, runs its experts, and
+ *     combines its own experts' rows per received token with tk_reduce into a bf16 partial;
+ *   - the source sums the partial rows of a token over its destination ranks in ascending
+ *     rank order, in fp32, rounded once to bf16 (tk_ep_combine).
+ * The kernels only read and write through the pointers given; on several GPUs those are peer
+ * addresses of the other ranks' buffers (the caller maps them, e.g. with symmetric memory) and
+ * the caller orders the phases across ranks (a collective between dispatch and the
+ * destinations' work, and between that and combine). No kernel waits on another rank.
+ */
+
+/* Bytes of device workspace tk_ep_layout needs. */
+TK_API size_t tk_ep_layout_workspace_bytes(int T, int G);
+
+/*
+ * Send layout of one source rank: the route map over destination ranks.
+ *   topk_idx      device, int32 [T, k] (expert -1 = masked pair: goes nowhere)
+ *   send_counts   device, int32 [G]: tokens this rank sends to each rank
+ *   send_offsets  device, int32 [G+1]: exclusive scan of send_counts
+ *   dest_slot     device, int32 [T, G]: send_offsets[d] + (position of token t among the tokens
+ *                 sent to d, in token order), or -1 when t does not go to d
+ *   send_token    device, int32 [T*G]: the token of each send row (rows past send_offsets[G]
+ *                 hold -1) -- a packed send buffer for a library all-to-all is
+ *                 tk_expand(x, dest_slot, send_offsets, send_token, T, G, G, ...)
+ *   workspace     device, tk_ep_layout_workspace_bytes(T, G) bytes, 16-byte aligned
+ *   err_flag      device int32 or NULL: TK_DEVERR_EXPERT_RANGE for an expert outside [0,E)
+ * 1 <= G <= TK_MAX_EP_RANKS, G divides E.
+ */
+TK_API tk_status tk_ep_layout(const int32_t* topk_idx, int T, int E, int k, int G,
+                              int32_t* send_counts, int32_t* send_offsets, int32_t* dest_slot,
+                              int32_t* send_token, void* workspace, size_t workspace_bytes,
+                              int32_t* err_flag, void* stream);
+
+/* One destination rank's receive buffers as seen from a source (device pointers, possibly a
+ * peer GPU's memory; all 16-byte aligned). */
+typedef struct tk_ep_peer {
+    void* x;          /* [rows, H]: bf16 rows, or E4M3 codes (one byte per channel) */
+    float* scale;     /* [rows, H/128] per-128-channel scales (E4M3 only; else NULL) */
+    int32_t* idx;     /* [rows, k] local expert ids, -1 for other ranks' experts */
+    float* w;         /* [rows, k] weights, 0 for other ranks' experts */
+    int64_t base_row; /* first row of this source's block in these buffers */
+    int64_t rows;     /* capacity of these buffers in rows (writes past it are skipped and
+                         flagged TK_DEVERR_ROWS_RANGE) */
+} tk_ep_peer;
+
+/*
+ * Dispatch of one source rank: every token row goes to each of its destination ranks, at row
+ * base_row + (dest_slot[t*G+d] - send_offsets[d]) of rank d's buffers, as bf16 or quantised on
+ * the way to E4M3 with per-128-channel scales (the same arithmetic as tk_expand's E4M3 path),
+ * with its k local expert ids and weights. One bulk load of each row, one bulk store per
+ * destination.
+ *   x             device, bf16 [T, H], 16-byte aligned;  topk_idx, topk_w  device [T, k]
+ *   dest_slot, send_offsets   from tk_ep_layout
+ *   peers         HOST array of G descriptors (copied into the launch; may be freed on return)
+ * H % 8 == 0 (H % 128 == 0 for E4M3).
+ */
+TK_API tk_status tk_ep_dispatch(const void* x, const int32_t* topk_idx, const float* topk_w,
+                                const int32_t* dest_slot, const int32_t* send_offsets, int T,
+                                int E, int k, int H, int G, int out_dtype, const tk_ep_peer* peers,
+                                int32_t* err_flag, void* stream);
+
+/*
+ * Combine of one source rank: out[t] = bf16( sum over ranks d ascending with
+ * dest_slot[t*G+d] >= 0 of fp32(partial[d][base_row[d] + dest_slot[t*G+d] - send_offsets[d]]) ),
+ * fp32 adds (a token that went nowhere gets zeros). partial[d] is rank d's bf16 [rows[d], H]
+ * buffer of per-received-row partial sums (tk_reduce over its local experts).
+ *   partial, base_row, rows   HOST arrays of G entries (partial[d]: device pointer, possibly a
+ *                 peer's memory, 16-byte aligned)
+ *   out           device, bf16 [T, H], 16-byte aligned
+ * A row index outside [0, rows[d]) is skipped and flagged TK_DEVERR_SLOT_RANGE.
+ */
+TK_API tk_status tk_ep_combine(const void* const* partial, const int64_t* base_row,
+                               const int64_t* rows, const int32_t* dest_slot,
+                               const int32_t* send_offsets, int T, int G, int H, void* out,
+                               int32_t* err_flag, void* stream);
 
 /*
  * Self-test of the library's bounded waits (no counterpart on the pages: it exists so that the

@@ -83,7 +83,7 @@ def test_route_map_rejects(tk):
         (dict(i=9, v=MISALIGNED), "aligned"),
         (dict(i=5, v=None), "NULL"),
         (dict(i=8, v=None), "token_of"),
-        (dict(i=3, v=17), "k"),
+        (dict(i=3, v=33), "k"),
     ]
     for change, what in bad:
         a = list(ok)
@@ -169,3 +169,41 @@ def test_selftest_rejects_bad_limits(tk):
     assert tk.lib.tk_selftest_bounded_wait(0, FAKE, None) == 1
     assert tk.lib.tk_selftest_bounded_wait(3_000_000_000, FAKE, None) == 1
     assert tk.lib.tk_selftest_bounded_wait(1000, None, None) == 1
+
+
+def test_ep_entries_reject_bad_arguments(tk):
+    L = tk.lib
+    T, G = 64, 4
+    ws = L.tk_ep_layout_workspace_bytes(T, G)
+    assert ws >= T * G * 4 and L.tk_ep_layout_workspace_bytes(T, 33) == 0
+    ok = [FAKE, T, 16, 2, G, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None, None]
+    for i, v, what in [(4, 0, "G="), (4, 33, "G="), (2, 18, "multiple of G"), (3, 33, "k="),
+                       (10, ws - 16, "workspace"), (9, MISALIGNED, "aligned"), (7, None, "NULL")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_ep_layout(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode(), what
+    peers = (tk.EpPeer * G)(*[tk.EpPeer(FAKE, None, FAKE, FAKE, 0, 100) for _ in range(G)])
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, T, 16, 2, 256, G, 0, peers, None, None]
+    for i, v, what in [(9, 33, "G="), (6, 18, "multiple of G"), (8, 12, "H="), (10, 5, "out_dtype"),
+                       (11, None, "peers"), (0, MISALIGNED, "aligned")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_ep_dispatch(*a) == 1, what
+        assert what in L.tk_last_error_detail().decode(), what
+    a = list(ok)
+    a[8], a[10] = 200, 1                   # E4M3 needs H % 128 == 0
+    assert L.tk_ep_dispatch(*a) == 1 and "128" in L.tk_last_error_detail().decode()
+    bad = (tk.EpPeer * G)(*[tk.EpPeer(None, None, FAKE, FAKE, 0, 100) for _ in range(G)])
+    a = list(ok)
+    a[11] = bad
+    assert L.tk_ep_dispatch(*a) == 1 and "receive buffers" in L.tk_last_error_detail().decode()
+    parts = (ctypes.c_void_p * G)(*[FAKE] * G)
+    base = (ctypes.c_int64 * G)(*[0] * G)
+    rows = (ctypes.c_int64 * G)(*[10] * G)
+    assert L.tk_ep_combine(parts, base, rows, FAKE, FAKE, T, 33, 256, FAKE, None, None) == 1
+    assert L.tk_ep_combine(parts, base, rows, FAKE, FAKE, T, G, 12, FAKE, None, None) == 1
+    assert L.tk_ep_combine(parts, base, rows, FAKE, FAKE, T, G, 256, MISALIGNED, None, None) == 1
+    neg = (ctypes.c_int64 * G)(*[-1] * G)
+    assert L.tk_ep_combine(parts, base, neg, FAKE, FAKE, T, G, 256, FAKE, None, None) == 1
+    assert L.tk_ep_combine(parts, base, rows, FAKE, FAKE, 0, G, 256, FAKE, None, None) == 0

@@ -1,0 +1,75 @@
+"""Host logic of the expert-parallel path, on CPU: the receive bases from the G x G send counts
+(against the oracle), and the count exchange between ranks over gloo -- every rank must end up
+with the same count matrix and bases, since each source writes into its peers' buffers at the
+base it computes itself."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def test_recv_bases_match_the_oracle(oracle_lib):
+    from token_routing_gate_b200 import ep
+
+    rng = np.random.default_rng(41)
+    for G in (1, 2, 3, 8, 32):
+        cm = rng.integers(0, 1000, (G, G)).astype(np.int32)
+        base, recv = ep.recv_bases(torch.from_numpy(cm))
+        o_base, o_recv = oracle_lib.ep_recv_bases(cm)
+        np.testing.assert_array_equal(base.numpy(), o_base)
+        np.testing.assert_array_equal(recv.numpy(), o_recv)
+    with pytest.raises(ValueError):
+        ep.recv_bases(torch.zeros(2, 3, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        ep.recv_bases(torch.tensor([[1, -1], [0, 0]]))
+    assert ep.capacity_rows(8192, 8) == 65536
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, result_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as tdist
+
+    import oracle
+    from token_routing_gate_b200 import dist, ep
+
+    assert dist.init("gloo", timeout_s=60)
+    E, k, T = 24, 4, 50 + 7 * rank          # ranks hold different numbers of tokens
+    rng = np.random.default_rng(100 + rank)
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, dest = oracle.ep_layout(idx, E, world)
+    cm = ep.exchange_counts(torch.from_numpy(counts))
+    base, recv = ep.recv_bases(cm)
+    np.testing.assert_array_equal(cm[rank].numpy(), counts)
+    gathered = [None] * world
+    tdist.all_gather_object(gathered, (counts, base.numpy(), recv.numpy(), idx))
+    if rank == 0:
+        for g in gathered:                  # one matrix, the same bases on every rank
+            np.testing.assert_array_equal(g[1], gathered[0][1])
+            np.testing.assert_array_equal(g[2], gathered[0][2])
+        o_base, o_recv = oracle.ep_recv_bases(np.stack([g[0] for g in gathered]))
+        np.testing.assert_array_equal(base.numpy(), o_base)
+        np.testing.assert_array_equal(recv.numpy(), o_recv)
+        # the blocks the sources write into each destination tile it exactly, without overlap
+        for d in range(world):
+            spans = sorted((int(o_base[s, d]), int(o_base[s, d]) + int(gathered[s][0][d]))
+                           for s in range(world))
+            assert spans[0][0] == 0 and spans[-1][1] == o_recv[d]
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+        open(os.path.join(result_dir, "ok"), "w").close()
+    dist.finish()
+
+
+def test_count_exchange_three_gloo_ranks(tmp_path, oracle_lib):
+    world = 3
+    mp.spawn(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    assert (tmp_path / "ok").exists()

@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "quant_e4m3.cuh"
 #include "tk_device.cuh"
 
 namespace tk {
@@ -47,8 +48,6 @@ __device__ __forceinline__ void store_copy(void* dst, const void* src, uint32_t 
 }
 constexpr int kFp8Threads = 256;
 constexpr int kFp8ChunkChannels = 8192;      // channels quantised per stage
-
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
 
 __global__ void __launch_bounds__(32)
 expand_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ slot_of, int k,
@@ -152,24 +151,7 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
         if (!load_ok) break;
         const int nb = chn / 128;
         for (int b = warp; b < nb; b += kFp8Threads / 32) {
-            const int cc = b * 128 + lane * 4;
-            const uint2 raw = *reinterpret_cast<const uint2*>(xin + cc);
-            const float f0 = bf16_bits_to_float(raw.x & 0xffffu);
-            const float f1 = bf16_bits_to_float(raw.x >> 16);
-            const float f2 = bf16_bits_to_float(raw.y & 0xffffu);
-            const float f3 = bf16_bits_to_float(raw.y >> 16);
-            const float a = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
-            // non-negative floats order like their bit patterns
-            const float amax = __uint_as_float(__reduce_max_sync(kFullMask, __float_as_uint(a)));
-            uint32_t q = 0u;
-            float scale = 0.0f;
-            if (amax != 0.0f) {
-                scale = __fdiv_rn(amax, 448.0f);
-                const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f0, scale), __fdiv_rn(f1, scale));
-                const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f2, scale), __fdiv_rn(f3, scale));
-                q = lo | (hi << 16);
-            }
-            *reinterpret_cast<uint32_t*>(qo + cc) = q;
+            const float scale = quantize_block_e4m3(xin + b * 128, qo + b * 128, lane);
             if (lane == 0) sc[b] = scale;
         }
         fence_proxy_async_smem();
@@ -203,8 +185,7 @@ extern "C" tk_status tk_expand(const void* x, const int32_t* slot_of, const int3
     using namespace tk;
     if (T < 0) return fail_arg("tk_expand: T=%d must be >= 0", T);
     if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_expand: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
-    if (k < 1 || k > E || k > TK_MAX_TOPK)
-        return fail_arg("tk_expand: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("tk_expand: k=%d outside [1, %d]", k, TK_MAX_TOPK);
     if (align < 1 || align > 4096) return fail_arg("tk_expand: align=%d outside [1, 4096]", align);
     if (out_dtype != TK_OUT_BF16 && out_dtype != TK_OUT_FP8_E4M3)
         return fail_arg("tk_expand: unknown out_dtype %d", out_dtype);

@@ -91,19 +91,22 @@ __device__ __forceinline__ void sort_desc(uint64_t (&v)[EPL]) {
     }
 }
 
-// One warp per token, tokens_per_warp consecutive tokens per warp (the grid is sized to one
-// wave of resident warps); the next token's logits are loaded while the current one is
-// processed. EPL = experts held per lane (E <= 32 * EPL).
+// One warp per token. The grid is one wave of resident warps and the T tokens are split evenly
+// over the nwarps warps (warp w takes tokens [w*T/nwarps, (w+1)*T/nwarps), so warps differ by
+// at most one token and every SM gets the same work); the next token's logits are loaded while
+// the current one is processed. EPL = experts held per lane (E <= 32 * EPL).
 template <int EPL>
 __global__ void __launch_bounds__(kGateWarps * 32)
 gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
-                 int k, int score_fn, int renormalize, int tokens_per_warp,
+                 int k, int score_fn, int renormalize, int nwarps,
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t t_begin = (static_cast<int64_t>(blockIdx.x) * kGateWarps + (threadIdx.x >> 5)) * tokens_per_warp;
-    if (t_begin >= T) return;
-    const int64_t t_end = min(static_cast<int64_t>(T), t_begin + tokens_per_warp);
+    const int64_t wid = static_cast<int64_t>(blockIdx.x) * kGateWarps + (threadIdx.x >> 5);
+    if (wid >= nwarps) return;
+    const int64_t t_begin = wid * T / nwarps;
+    const int64_t t_end = (wid + 1) * T / nwarps;
+    if (t_begin >= t_end) return;
 
     float b[EPL];  // this lane's selection biases, shared by all tokens
 #pragma unroll
@@ -205,7 +208,7 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
 template <int EPL>
 cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, int k, int score_fn,
                         int renormalize, int32_t* idx, float* w, cudaStream_t s) {
-    // one wave: as many warps as fit on the GPU at once, each taking consecutive tokens
+    // one wave: as many warps as fit on the GPU at once, each taking a run of consecutive tokens
     static std::atomic<int> resident[kMaxDevices];
     const int dev = current_device();
     int resident_warps = resident[dev].load(std::memory_order_acquire);
@@ -217,11 +220,10 @@ cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, in
         resident_warps = per_sm * kGateWarps * num_sms();
         resident[dev].store(resident_warps, std::memory_order_release);
     }
-    const int tpw = (T + resident_warps - 1) / resident_warps;
-    const int warps = (T + tpw - 1) / tpw;
+    const int warps = min(T, resident_warps);
     const dim3 grid((warps + kGateWarps - 1) / kGateWarps);
     return launch_pdl(gate_topk_kernel<EPL>, grid, dim3(kGateWarps * 32), 0, s, logits, bias, T, E,
-                      k, score_fn, renormalize, tpw, idx, w);
+                      k, score_fn, renormalize, warps, idx, w);
 }
 
 }  // namespace

@@ -81,10 +81,68 @@ size_t smem_bytes(int k, int S) {
            static_cast<size_t>(2 * S) * sizeof(uint64_t);
 }
 
+// Where the j-th row of token t comes from. fetch() reads the pair's index (one unit ahead of
+// use); lane_ctx() caches what lane j needs to resolve it; resolve() gives the row's address,
+// or nullptr for a row that does not exist (flagging an index that is not a valid one).
+//
+// SlotRows (the reduce): row j of token t is y[slot_of[t*k + j]]; slot -1 is a masked pair.
+struct SlotRows {
+    const uint8_t* y;
+    int64_t y_rows;
+    const int32_t* slot_of;
+    struct Lane {};
+    __device__ __forceinline__ Lane lane_ctx(int) const { return {}; }
+    __device__ __forceinline__ int64_t fetch(int64_t t, int j, int k) const { return slot_of[t * k + j]; }
+    __device__ __forceinline__ const uint8_t* resolve(const Lane&, int64_t raw, int64_t row_bytes,
+                                                      int32_t* err) const {
+        if (raw >= 0 && raw < y_rows) return y + raw * row_bytes;
+        if (raw != -1) flag_error(err, TK_DEVERR_SLOT_RANGE);
+        return nullptr;
+    }
+};
+
+// RankRows (the expert-parallel combine): "row j" of token t is the partial row rank j holds
+// for it, at base[j] + (dest_slot[t*G + j] - send_offsets[j]) in rank j's partial buffer
+// (dest_slot -1: the token did not go to rank j).
+struct RankRows {
+    const uint8_t* part[TK_MAX_EP_RANKS];
+    int64_t base[TK_MAX_EP_RANKS];
+    int64_t rows[TK_MAX_EP_RANKS];
+    const int32_t* dest_slot;
+    const int32_t* send_offsets;
+    int G;
+    struct Lane {
+        const uint8_t* part;
+        int64_t base, rows;
+        int32_t off;
+    };
+    __device__ __forceinline__ Lane lane_ctx(int j) const {
+        Lane L{nullptr, 0, 0, 0};
+        if (j < G) {
+            L.part = part[j];
+            L.base = base[j];
+            L.rows = rows[j];
+            L.off = send_offsets[j];
+        }
+        return L;
+    }
+    __device__ __forceinline__ int64_t fetch(int64_t t, int j, int) const { return dest_slot[t * G + j]; }
+    __device__ __forceinline__ const uint8_t* resolve(const Lane& L, int64_t raw, int64_t row_bytes,
+                                                      int32_t* err) const {
+        if (raw == -1) return nullptr;
+        const int64_t row = L.base + (raw - L.off);
+        if (raw < 0 || raw < L.off || row >= L.rows) {
+            flag_error(err, TK_DEVERR_SLOT_RANGE);
+            return nullptr;
+        }
+        return L.part + row * row_bytes;
+    }
+};
+
+template <class Rows>
 __global__ void __launch_bounds__(kRedThreads)
-reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __restrict__ slot_of,
-              const float* __restrict__ w, int T, int k, int H, int S, uint8_t* __restrict__ out,
-              int32_t* err_flag) {
+reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, int T, int k, int H,
+              int S, uint8_t* __restrict__ out, int32_t* err_flag) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int stage_bytes = k * kChunkBytes;
     uint8_t* data = sm;
@@ -110,12 +168,13 @@ reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __re
     if (warp == 0) {
         // ---------------- producer (slots and weights of the next unit are fetched while the
         // current unit waits for a free stage)
+        const typename Rows::Lane lctx = rows.lane_ctx(lane);
         int64_t u = blockIdx.x;
         int64_t nxt_sl = -1;
         float nxt_w = 1.0f;
         if (lane < k && u < units) {
             const int64_t t = u / chunks;
-            nxt_sl = slot_of[t * k + lane];
+            nxt_sl = rows.fetch(t, lane, k);
             if (w != nullptr) nxt_w = w[t * k + lane];
         }
         for (int it = 0; u < units; u += gridDim.x, ++it) {
@@ -129,14 +188,10 @@ reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __re
             const int64_t un = u + gridDim.x;
             if (lane < k && un < units) {
                 const int64_t tn = un / chunks;
-                nxt_sl = slot_of[tn * k + lane];
+                nxt_sl = rows.fetch(tn, lane, k);
                 if (w != nullptr) nxt_w = w[tn * k + lane];
             }
-            int64_t sl = -1;
-            if (lane < k) {
-                if (raw >= 0 && raw < y_rows) sl = raw;
-                else if (raw != -1) flag_error(err_flag, TK_DEVERR_SLOT_RANGE);
-            }
+            const uint8_t* rowp = lane < k ? rows.resolve(lctx, raw, row_bytes, err_flag) : nullptr;
             int ok = 1;
             if (lane == 0) ok = mbar_wait_bounded(&empty[s], ph ^ 1u) ? 1 : 0;
             ok = __shfl_sync(kFullMask, ok, 0);
@@ -146,15 +201,15 @@ reduce_kernel(const uint8_t* __restrict__ y, int64_t y_rows, const int32_t* __re
             }
             if (lane < k) {
                 meta[s].w[lane] = wl;
-                meta[s].valid[lane] = sl >= 0 ? 1 : 0;
+                meta[s].valid[lane] = rowp != nullptr ? 1 : 0;
             }
-            const unsigned vmask = __ballot_sync(kFullMask, sl >= 0);
+            const unsigned vmask = __ballot_sync(kFullMask, rowp != nullptr);
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(vmask)) * bytes);
             __syncwarp();
-            if (sl >= 0) {
+            if (rowp != nullptr) {
                 uint8_t* dst = data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * kChunkBytes;
-                const uint8_t* src = y + sl * row_bytes + static_cast<int64_t>(ch0) * 2;
+                const uint8_t* src = rowp + static_cast<int64_t>(ch0) * 2;
                 if (TK_REDUCE_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, &full[s], l2_policy(TK_REDUCE_LOAD_POLICY));
                 else bulk_load(dst, src, bytes, &full[s]);
             }
@@ -212,8 +267,9 @@ struct LaunchShape {
     int S = 0;
 };
 
-// Launch shape for k on the current device, worked out once (the kernel's shared-memory limit
-// is raised to the largest size any k needs).
+// Launch shape for k on the current device, worked out once per row source (the kernel's
+// shared-memory limit is raised to the largest size any k needs).
+template <class Rows>
 cudaError_t launch_shape(int k, LaunchShape& out) {
     static LaunchShape shapes[kMaxDevices][TK_MAX_TOPK + 1];
     static std::atomic<bool> ready[kMaxDevices][TK_MAX_TOPK + 1];
@@ -229,13 +285,13 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
         const size_t smem = smem_bytes(k, S);
         cudaError_t err = cudaSuccess;
         if (static_cast<int>(smem) > configured_smem[dev]) {
-            err = cudaFuncSetAttribute(reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(reduce_kernel<Rows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
             if (err != cudaSuccess) return err;
             configured_smem[dev] = static_cast<int>(smem);
         }
         int per_sm = 0;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel, kRedThreads, smem);
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows>, kRedThreads, smem);
         if (err != cudaSuccess) return err;
         shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
         shapes[dev][k].S = S;
@@ -243,6 +299,22 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
     }
     out = shapes[dev][k];
     return cudaSuccess;
+}
+
+template <class Rows>
+cudaError_t launch_reduce(const Rows& rows, const float* w, int T, int k, int H, void* out,
+                          int32_t* err_flag, void* stream, const char** what) {
+    *what = "reduce_kernel setup";
+    LaunchShape shape;
+    const cudaError_t e = launch_shape<Rows>(k, shape);
+    if (e != cudaSuccess) return e;
+    *what = "reduce_kernel";
+    const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
+    const int64_t units = static_cast<int64_t>(T) * chunks;
+    const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);
+    return launch_pdl(reduce_kernel<Rows>, dim3(grid), dim3(kRedThreads), smem_bytes(k, shape.S),
+                      static_cast<cudaStream_t>(stream), rows, w, T, k, H, shape.S,
+                      static_cast<uint8_t*>(out), err_flag);
 }
 
 }  // namespace
@@ -260,15 +332,38 @@ extern "C" tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slo
         return fail_arg("tk_reduce: y, slot_of and out must not be NULL");
     if (reinterpret_cast<uintptr_t>(y) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 16 != 0)
         return fail_arg("tk_reduce: y and out must be 16-byte aligned");
-    LaunchShape shape;
-    const cudaError_t e = launch_shape(k, shape);
-    if (e != cudaSuccess) return check_launch(e, "reduce_kernel setup");
-    const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
-    const int64_t units = static_cast<int64_t>(T) * chunks;
-    const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);
-    cudaError_t err = launch_pdl(reduce_kernel, dim3(grid), dim3(kRedThreads),
-                                 smem_bytes(k, shape.S), static_cast<cudaStream_t>(stream),
-                                 static_cast<const uint8_t*>(y), y_rows, slot_of, w, T, k, H,
-                                 shape.S, static_cast<uint8_t*>(out), err_flag);
-    return check_launch(err, "reduce_kernel");
+    const SlotRows rows{static_cast<const uint8_t*>(y), y_rows, slot_of};
+    const char* what = "";
+    const cudaError_t err = launch_reduce(rows, w, T, k, H, out, err_flag, stream, &what);
+    return check_launch(err, what);
+}
+
+extern "C" tk_status tk_ep_combine(const void* const* partial, const int64_t* base_row,
+                                   const int64_t* rows, const int32_t* dest_slot,
+                                   const int32_t* send_offsets, int T, int G, int H, void* out,
+                                   int32_t* err_flag, void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_ep_combine: T=%d must be >= 0", T);
+    if (G < 1 || G > TK_MAX_EP_RANKS) return fail_arg("tk_ep_combine: G=%d outside [1, %d]", G, TK_MAX_EP_RANKS);
+    if (H < 8 || H % 8 != 0) return fail_arg("tk_ep_combine: H=%d must be a positive multiple of 8", H);
+    if (T == 0) return TK_OK;
+    if (partial == nullptr || base_row == nullptr || rows == nullptr || dest_slot == nullptr ||
+        send_offsets == nullptr || out == nullptr)
+        return fail_arg("tk_ep_combine: no pointer argument may be NULL");
+    if (reinterpret_cast<uintptr_t>(out) % 16 != 0) return fail_arg("tk_ep_combine: out must be 16-byte aligned");
+    RankRows rr{};
+    for (int d = 0; d < G; ++d) {
+        if (rows[d] < 0 || base_row[d] < 0) return fail_arg("tk_ep_combine: rank %d has negative rows or base", d);
+        if (rows[d] > 0 && (partial[d] == nullptr || reinterpret_cast<uintptr_t>(partial[d]) % 16 != 0))
+            return fail_arg("tk_ep_combine: partial[%d] must be a 16-byte aligned buffer", d);
+        rr.part[d] = static_cast<const uint8_t*>(partial[d]);
+        rr.base[d] = base_row[d];
+        rr.rows[d] = rows[d];
+    }
+    rr.dest_slot = dest_slot;
+    rr.send_offsets = send_offsets;
+    rr.G = G;
+    const char* what = "";
+    const cudaError_t err = launch_reduce(rr, nullptr, T, G, H, out, err_flag, stream, &what);
+    return check_launch(err, what);
 }

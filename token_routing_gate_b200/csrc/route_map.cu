@@ -340,8 +340,7 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
     using namespace tk;
     if (T < 0) return fail_arg("tk_route_map: T=%d must be >= 0", T);
     if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_route_map: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
-    if (k < 1 || k > E || k > TK_MAX_TOPK)
-        return fail_arg("tk_route_map: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("tk_route_map: k=%d outside [1, %d]", k, TK_MAX_TOPK);
     if (align < 1 || align > 4096) return fail_arg("tk_route_map: align=%d outside [1, 4096]", align);
     const int64_t rmax = tk_max_rows(T, E, k, align);
     if (rmax > INT32_MAX) return fail_arg("tk_route_map: T*k + E*(align-1) = %lld exceeds int32", (long long)rmax);
@@ -436,8 +435,7 @@ extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, 
     if (T < 0) return fail_arg("tk_route_map_static: T=%d must be >= 0", T);
     if (E < 1 || E > TK_MAX_EXPERTS)
         return fail_arg("tk_route_map_static: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
-    if (k < 1 || k > E || k > TK_MAX_TOPK)
-        return fail_arg("tk_route_map_static: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("tk_route_map_static: k=%d outside [1, %d]", k, TK_MAX_TOPK);
     if (align < 1 || align > 4096)
         return fail_arg("tk_route_map_static: align=%d outside [1, 4096]", align);
     const int64_t rmax = tk_max_rows(T, E, k, align);

@@ -27,8 +27,15 @@ DEVERR_TIMEOUT = 16
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
                "tk_route_map_static", "tk_expand", "tk_reduce", "tk_balance_stats_workspace_bytes",
                "tk_balance_stats", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
-               "tk_reduce_backward", "tk_expand_backward", "tk_selftest_bounded_wait", "tk_status_str",
-               "tk_last_error_detail", "tk_abi_version")
+               "tk_reduce_backward", "tk_expand_backward", "tk_ep_layout_workspace_bytes",
+               "tk_ep_layout", "tk_ep_dispatch", "tk_ep_combine", "tk_selftest_bounded_wait",
+               "tk_status_str", "tk_last_error_detail", "tk_abi_version")
+
+
+class EpPeer(ctypes.Structure):
+    """tk_ep_peer: one destination rank's receive buffers (device addresses)."""
+    _fields_ = [("x", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+                ("w", ctypes.c_void_p), ("base_row", ctypes.c_int64), ("rows", ctypes.c_int64)]
 
 
 class TkError(RuntimeError):
@@ -72,6 +79,16 @@ def _load():
     L.tk_reduce_backward.restype = i32
     L.tk_expand_backward.argtypes = [vp, i64, vp, i32, i32, i32, vp, vp, vp]
     L.tk_expand_backward.restype = i32
+    L.tk_ep_layout_workspace_bytes.argtypes = [i32, i32]
+    L.tk_ep_layout_workspace_bytes.restype = sz
+    L.tk_ep_layout.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.tk_ep_layout.restype = i32
+    L.tk_ep_dispatch.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                 ctypes.POINTER(EpPeer), vp, vp]
+    L.tk_ep_dispatch.restype = i32
+    L.tk_ep_combine.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int64),
+                                ctypes.POINTER(ctypes.c_int64), vp, vp, i32, i32, i32, vp, vp, vp]
+    L.tk_ep_combine.restype = i32
     L.tk_selftest_bounded_wait.argtypes = [i64, vp, vp]
     L.tk_selftest_bounded_wait.restype = i32
     L.tk_status_str.argtypes = [i32]
@@ -247,3 +264,74 @@ def selftest_bounded_wait(limit_ns, err_flag, stream=None):
     """Run the bounded-wait self-test kernel (it always times out and flags DEVERR_TIMEOUT)."""
     _check("tk_selftest_bounded_wait", lib.tk_selftest_bounded_wait(int(limit_ns), _ptr(err_flag),
                                                                     _stream(stream)))
+
+
+# ---------------------------------------------------------------- expert-parallel dispatch / combine
+def _addr(t):
+    """Device address of a tensor (contiguous) or a raw integer address (e.g. a peer's buffer)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libtk_route must be contiguous")
+    return t.data_ptr()
+
+
+class EpLayout:
+    """Send layout of one source rank (tk_ep_layout): the route map over destination ranks."""
+
+    def __init__(self, send_counts, send_offsets, dest_slot, send_token, workspace, G):
+        self.send_counts, self.send_offsets = send_counts, send_offsets
+        self.dest_slot, self.send_token, self.workspace, self.G = dest_slot, send_token, workspace, G
+
+
+def ep_layout(topk_idx, E, G, out=None, err_flag=None, stream=None):
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if out is None:
+        out = EpLayout(torch.empty(G, dtype=torch.int32, device=dev),
+                       torch.empty(G + 1, dtype=torch.int32, device=dev),
+                       torch.empty(T, G, dtype=torch.int32, device=dev),
+                       torch.empty(T * G, dtype=torch.int32, device=dev),
+                       _workspace(int(lib.tk_ep_layout_workspace_bytes(T, G)), dev), G)
+    _check("tk_ep_layout", lib.tk_ep_layout(
+        _ptr(topk_idx), T, E, k, G, _ptr(out.send_counts), _ptr(out.send_offsets),
+        _ptr(out.dest_slot), _ptr(out.send_token), _ptr(out.workspace), out.workspace.numel(),
+        _ptr(err_flag), _stream(stream)))
+    return out
+
+
+def ep_peer(x, idx, w, base_row, rows, scale=None):
+    """Descriptor of one destination's receive buffers: tensors or raw device addresses."""
+    return EpPeer(_addr(x), _addr(scale), _addr(idx), _addr(w), int(base_row), int(rows))
+
+
+def ep_dispatch(x, topk_idx, topk_w, layout, E, peers, out_dtype="bf16", err_flag=None,
+                stream=None):
+    """Writes this rank's tokens into the G destinations' receive buffers (peers: G EpPeer)."""
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    G = layout.G
+    if len(peers) != G:
+        raise ValueError(f"{len(peers)} peer descriptors for G={G}")
+    arr = (EpPeer * G)(*peers)
+    _check("tk_ep_dispatch", lib.tk_ep_dispatch(
+        _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(layout.dest_slot), _ptr(layout.send_offsets),
+        T, E, k, H, G, OUT_DTYPE[out_dtype], arr, _ptr(err_flag), _stream(stream)))
+
+
+def ep_combine(partials, base_rows, rows, layout, H, out=None, err_flag=None, stream=None):
+    """out[t] = bf16(sum over destinations d ascending of partials[d][base_rows[d] + position]).
+    partials: G tensors or raw device addresses of bf16 [rows[d], H] buffers."""
+    G = layout.G
+    T = layout.dest_slot.shape[0]
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=layout.dest_slot.device)
+    ptrs = (ctypes.c_void_p * G)(*[_addr(p) for p in partials])
+    base = (ctypes.c_int64 * G)(*[int(b) for b in base_rows])
+    nrows = (ctypes.c_int64 * G)(*[int(r) for r in rows])
+    _check("tk_ep_combine", lib.tk_ep_combine(
+        ptrs, base, nrows, _ptr(layout.dest_slot), _ptr(layout.send_offsets), T, G, H, _ptr(out),
+        _ptr(err_flag), _stream(stream)))
+    return out
