@@ -574,6 +574,27 @@ def run_ep(args, wl):
     prev = ["start"] + names[:-1]
     phase_us = {n: 1e3 * sum(e[p].elapsed_time(e[n]) for e in evs) / K for p, n in zip(prev, names)}
     step_ms = sum(e["start"].elapsed_time(e["combine"]) for e in evs) / K
+    # the dispatch and combine kernels on their own: rank 0's call launched back to back
+    lay0 = res["layouts"][0]
+    base0 = res["base"][0]
+    peers0 = [vr.bufs[d].peer(int(base0[d])) for d in range(G)]
+    kernel_us = {}
+    for name, fn in (("dispatch", lambda: tk.ep_dispatch(xs[0], idxs[0], ws[0], lay0, E, peers0,
+                                                         args.ep_dtype, stream=stream)),
+                     ("combine", lambda: tk.ep_combine([b.partial for b in vr.bufs], base0.tolist(),
+                                                       recv.tolist(), lay0, H, out=outs[0],
+                                                       stream=stream))):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(K):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        kernel_us[name] = 1e3 * a.elapsed_time(b) / K
+    sent0 = int(lay0.send_counts.sum())
     sent_rows = int(recv.sum())
     row_out = H if args.ep_dtype == "fp8" else 2 * H
     scale_b = 4 * (H // 128) if args.ep_dtype == "fp8" else 0
@@ -587,6 +608,10 @@ def run_ep(args, wl):
                        "tokens_per_rank": Tr, "rows_sent": sent_rows,
                        "emulated": "all ranks on one GPU: transfers are local HBM traffic"},
             "phases_us": phase_us,
+            "kernel_us": kernel_us,
+            "kernel_gbs": {"dispatch": (Tr * 2 * H + sent0 * (row_out + scale_b + 8 * k) + Tr * k * 8)
+                           / (kernel_us["dispatch"] * 1e3),
+                           "combine": (sent0 * 2 * H + Tr * 2 * H) / (kernel_us["combine"] * 1e3)},
             "hbm_gbs": {"dispatch": disp_bytes / (phase_us["dispatch"] * 1e3),
                         "combine": comb_bytes / (phase_us["combine"] * 1e3)},
             "bytes": {"dispatch": disp_bytes, "combine": comb_bytes},

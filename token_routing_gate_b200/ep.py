@@ -97,13 +97,27 @@ class VirtualRanks:
         self.out_dtype = out_dtype
         self.capacity = capacity_rows(max_tokens, G)
         self.bufs = [RankBuffers(self.capacity, H, k, out_dtype, device) for _ in range(G)]
+        self._layouts = {}   # (rank, T) -> preallocated layout outputs
+
+    def _layout_out(self, s, T, device):
+        key = (s, T)
+        if key not in self._layouts:
+            G = self.G
+            self._layouts[key] = tk.EpLayout(
+                torch.empty(G, dtype=torch.int32, device=device),
+                torch.empty(G + 1, dtype=torch.int32, device=device),
+                torch.empty(T, G, dtype=torch.int32, device=device),
+                torch.empty(T * G, dtype=torch.int32, device=device),
+                tk._workspace(int(tk.lib.tk_ep_layout_workspace_bytes(T, G)), device), G)
+        return self._layouts[key]
 
     def step(self, xs, idxs, ws, expert_fn, outs=None, err_flag=None, stream=None, mark=None):
         """One step of all G ranks. mark(name), if given, is called at the phase boundaries
         ("layout", "dispatch", "experts", "combine": the end of each phase)."""
         G = self.G
         mark = mark or (lambda name: None)
-        layouts = [tk.ep_layout(idxs[s], self.E, G, err_flag=err_flag, stream=stream) for s in range(G)]
+        layouts = [tk.ep_layout(idxs[s], self.E, G, out=self._layout_out(s, idxs[s].shape[0], idxs[s].device),
+                                err_flag=err_flag, stream=stream) for s in range(G)]
         cm = torch.stack([lay.send_counts for lay in layouts]).cpu()      # the count exchange
         base, recv_rows = recv_bases(cm)
         if int(recv_rows.max()) > self.capacity:
