@@ -48,6 +48,9 @@ def parse_args():
                         "expert-parallel dispatch/combine of the batch over --ep-ranks ranks run "
                         "on one GPU")
     p.add_argument("--ep-ranks", type=int, default=8, help="ranks of the --op ep run")
+    p.add_argument("--ep-tokens", type=int, default=None,
+                   help="tokens per rank of the --op ep run (default: the workload's T, i.e. every "
+                        "rank holds one 8K-token batch, the pages' EP setting)")
     p.add_argument("--ep-dtype", choices=["bf16", "fp8"], default="fp8",
                    help="dispatch format of the --op ep run (the pages' setting: FP8 dispatch)")
     return p.parse_args()
@@ -522,9 +525,10 @@ def run_op(args, wl):
 
 
 def run_ep(args, wl):
-    """Expert-parallel dispatch -> experts' combine -> combine of the workload's batch split over
-    G ranks, all run on one GPU (VirtualRanks). The "transfers" are writes and reads of this
-    GPU's own memory, so the numbers are HBM numbers of the EP kernels, not NVLink numbers."""
+    """Expert-parallel dispatch -> experts' combine -> combine over G ranks that each hold
+    --ep-tokens tokens of the workload's shape, all run on one GPU (VirtualRanks). The
+    "transfers" are writes and reads of this GPU's own memory, so the numbers are HBM numbers of
+    the EP kernels, not NVLink numbers."""
     import torch
     from token_routing_gate_b200 import ep, tk
     from token_routing_gate_b200 import workloads as W
@@ -533,10 +537,12 @@ def run_ep(args, wl):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     G = args.ep_ranks
-    T, E, k, H = wl.T, wl.E, wl.k, wl.H
-    if T % G or E % G:
-        raise SystemExit(f"--ep-ranks {G} must divide T={T} and E={E}")
-    Tr = T // G
+    Tr = args.ep_tokens or wl.T
+    E, k, H = wl.E, wl.k, wl.H
+    T = Tr * G
+    if E % G:
+        raise SystemExit(f"--ep-ranks {G} must divide E={E}")
+    wl = wl.with_(T=T)
     logits, bias = W.gate_inputs(wl, dev)
     x = W.activations(wl, dev)
     idx, w = tk.gate_topk(logits, k, wl.score, bias)
@@ -578,6 +584,9 @@ def run_ep(args, wl):
     lay0 = res["layouts"][0]
     base0 = res["base"][0]
     peers0 = [vr.bufs[d].peer(int(base0[d])) for d in range(G)]
+    # (one launch moves less than the 126 MB L2, so L2 is flushed before every timed launch by
+    # writing a 256 MB buffer, and each launch is timed on its own)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     kernel_us = {}
     for name, fn in (("dispatch", lambda: tk.ep_dispatch(xs[0], idxs[0], ws[0], lay0, E, peers0,
                                                          args.ep_dtype, stream=stream)),
@@ -586,14 +595,16 @@ def run_ep(args, wl):
                                                        stream=stream))):
         for _ in range(3):
             fn()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(K)]
         torch.cuda.synchronize(dev)
-        a.record(stream)
-        for _ in range(K):
+        for a, b in pairs:
+            flush.fill_(1)
+            a.record(stream)
             fn()
-        b.record(stream)
+            b.record(stream)
         torch.cuda.synchronize(dev)
-        kernel_us[name] = 1e3 * a.elapsed_time(b) / K
+        kernel_us[name] = 1e3 * sum(a.elapsed_time(b) for a, b in pairs) / K
     sent0 = int(lay0.send_counts.sum())
     sent_rows = int(recv.sum())
     row_out = H if args.ep_dtype == "fp8" else 2 * H
@@ -604,7 +615,8 @@ def run_ep(args, wl):
             "op": "ep", "value": T / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
             "dtype": args.ep_dtype, "data": "synthetic",
-            "config": {"workload": wl.name, "T": T, "E": E, "k": k, "H": H, "ranks": G,
+            "config": {"workload": f"ep{G}_T{Tr}_per_rank_E{E}_k{k}_H{H}_{wl.score}"
+                                   + ("_bias" if wl.bias else ""), "T": T, "E": E, "k": k, "H": H, "ranks": G,
                        "tokens_per_rank": Tr, "rows_sent": sent_rows,
                        "emulated": "all ranks on one GPU: transfers are local HBM traffic"},
             "phases_us": phase_us,
