@@ -5,17 +5,21 @@
 // Pure bandwidth: per token, k scattered 2H-byte rows read and one 2H-byte row written. The
 // loads go through the bulk-copy (TMA) engine so that the bytes in flight do not depend on
 // registers: a unit of work is (token t, 1024-channel chunk c). Each CTA is warp-specialised:
-//   warp 0      producer: lanes j < k read slot j and weight j of the unit, park the weights in
-//               the stage's shared-memory header, and issue one 1-D bulk load per valid row
-//               chunk (2 KB each) into the stage, completing on the stage's "full" mbarrier
-//               (transaction count = bytes issued).
+//   warp 0      producer: lanes j < k read slot j and weight j of the unit, and the unit's valid
+//               rows (masked pairs and absent rows skipped) get consecutive 2 KB places in a
+//               shared-memory byte ring, in slot order; their weights go to the unit's entry
+//               (one of 16), and one 1-D bulk load per valid row chunk completes on the entry's
+//               "full" mbarrier (transaction count = bytes issued).
 //   warps 1..4  consumers: wait "full", each thread combines one 8-channel vector of the unit
-//               across the k row chunks (16-byte shared loads, fmaf in slot order), writes 16
-//               bytes of bf16 output, then the warp arrives on the stage's "empty" mbarrier.
-// The ring has S stages with S*k*2 KB <= 32 KB (two at k = 8), so an SM holds about six CTAs and
-// up to ~190 KB of loads in flight. A measured sweep on B200 (ring depth, chunk width, consumer
-// warps) put this shape at the HBM copy roofline; deeper rings with fewer CTAs per SM were up to
-// 30% slower. The grid is persistent (SM count x CTAs per SM) and CTAs stride over units.
+//               across its valid row chunks (16-byte shared loads, fmaf in slot order), writes
+//               16 bytes of bf16 output, then the warp arrives on the entry's "empty" mbarrier.
+// The ring holds 32 KB, so a unit whose k = 8 rows are all valid takes 16 KB (two in flight, as a
+// fixed two-stage ring would), while a unit with few valid rows -- a masked route map, an
+// expert-parallel destination's rows -- takes only what it loads and up to 16 units are in
+// flight. About six CTAs fit on an SM (~190 KB of loads in flight). A measured sweep on B200
+// (ring size, chunk width, consumer warps) put this shape at the HBM copy roofline; deeper rings
+// with fewer CTAs per SM were up to 30% slower. The grid is persistent (SM count x CTAs per SM)
+// and CTAs stride over units.
 // The row loads carry an explicit L2 evict-normal policy. Measured on B200 at T=8192, H=7168,
 // k=8: with it the reduce after dispatch and the reduce run back to back were both faster than
 // with no policy operand (forward step 366.8 -> 364.9 us; back-to-back reduce 155.5 -> 152.9 us).
@@ -49,11 +53,14 @@ constexpr int kRedThreads = 32 * (1 + kConsumerWarps);
 constexpr int kChunkCh = 8 * 32 * kConsumerWarps * kVecs;  // channels per unit
 constexpr int kChunkBytes = kChunkCh * 2;                  // bf16 bytes of one row chunk
 constexpr int kStageBudget = TK_REDUCE_STAGE_KB * 1024;    // shared bytes of row data per CTA
-constexpr int kMaxStages = 8;
+constexpr int kRingEntries = 16;                           // units in flight at most
 
-struct StageMeta {
+// One unit's entry in the ring: its valid rows sit back to back at `off`, in slot order, and
+// w[i] is the weight of the i-th of them.
+struct EntryMeta {
     float w[TK_MAX_TOPK];
-    int32_t valid[TK_MAX_TOPK];
+    int32_t n;
+    uint32_t off;
 };
 
 __device__ __forceinline__ float lo_bf16(uint32_t v) { return __uint_as_float(v << 16); }
@@ -65,20 +72,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return l | (h << 16);
 }
 
-int stages_for(int k) {
-#ifdef TK_REDUCE_STAGES
-    (void)k;
-    return TK_REDUCE_STAGES;
-#endif
-    int s = kStageBudget / (k * kChunkBytes);
-    if (s < 1) s = 1;
-    if (s > kMaxStages) s = kMaxStages;
-    return s;
-}
+// Bytes of the row ring: the budget, and at least one unit with all k rows valid.
+int ring_bytes_for(int k) { return k * kChunkBytes > kStageBudget ? k * kChunkBytes : kStageBudget; }
 
-size_t smem_bytes(int k, int S) {
-    return static_cast<size_t>(S) * k * kChunkBytes + static_cast<size_t>(S) * sizeof(StageMeta) +
-           static_cast<size_t>(2 * S) * sizeof(uint64_t);
+size_t smem_bytes(int ring) {
+    return static_cast<size_t>(ring) + kRingEntries * sizeof(EntryMeta) +
+           2 * kRingEntries * sizeof(uint64_t);
 }
 
 // Where the j-th row of token t comes from. fetch() reads the pair's index (one unit ahead of
@@ -142,19 +141,18 @@ struct RankRows {
 template <class Rows>
 __global__ void __launch_bounds__(kRedThreads)
 reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, int T, int k, int H,
-              int S, uint8_t* __restrict__ out, int32_t* err_flag) {
+              int ring, uint8_t* __restrict__ out, int32_t* err_flag) {
     extern __shared__ __align__(128) uint8_t sm[];
-    const int stage_bytes = k * kChunkBytes;
-    uint8_t* data = sm;
-    StageMeta* meta = reinterpret_cast<StageMeta*>(sm + static_cast<size_t>(S) * stage_bytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(meta + S);
-    uint64_t* empty = full + S;
+    uint8_t* data = sm;                                                    // [ring] row bytes
+    EntryMeta* meta = reinterpret_cast<EntryMeta*>(sm + ring);             // [kRingEntries]
+    uint64_t* full = reinterpret_cast<uint64_t*>(meta + kRingEntries);
+    uint64_t* empty = full + kRingEntries;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+        for (int e = 0; e < kRingEntries; ++e) {
+            mbar_init(&full[e], 1);
+            mbar_init(&empty[e], kConsumerWarps);
         }
         fence_barrier_init();
     }
@@ -166,8 +164,11 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
     const int64_t row_bytes = static_cast<int64_t>(H) * 2;
 
     if (warp == 0) {
-        // ---------------- producer (slots and weights of the next unit are fetched while the
-        // current unit waits for a free stage)
+        // ---------------- producer. Unit `it` takes entry it % kRingEntries and the next
+        // (valid rows) * 2 KB of the ring (wrapping to its start when the rest of the ring is
+        // too short). Before reusing space or an entry it waits, oldest first, for the
+        // consumers to release earlier units; lane e remembers where entry e's bytes end.
+        // The slots and weights of the next unit are fetched while the current one waits.
         const typename Rows::Lane lctx = rows.lane_ctx(lane);
         int64_t u = blockIdx.x;
         int64_t nxt_sl = -1;
@@ -177,9 +178,10 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
             nxt_sl = rows.fetch(t, lane, k);
             if (w != nullptr) nxt_w = w[t * k + lane];
         }
+        uint64_t head = 0, tail = 0;   // ring bytes handed out / released so far
+        uint64_t my_end = 0;           // lane e: end of entry e's bytes
+        int rel = 0;                   // units known to be released
         for (int it = 0; u < units; u += gridDim.x, ++it) {
-            const int s = it % S;
-            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
             const int64_t t = u / chunks;
             const int ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
             const uint32_t bytes = static_cast<uint32_t>(min(kChunkCh, H - ch0)) * 2u;
@@ -192,26 +194,46 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
                 if (w != nullptr) nxt_w = w[tn * k + lane];
             }
             const uint8_t* rowp = lane < k ? rows.resolve(lctx, raw, row_bytes, err_flag) : nullptr;
+            const unsigned vmask = __ballot_sync(kFullMask, rowp != nullptr);
+            const int nvalid = __popc(vmask);
+            const int pos = __popc(vmask & ((1u << lane) - 1u));   // this row's place among them
+            uint64_t h = head;
+            uint32_t off = static_cast<uint32_t>(h % static_cast<uint64_t>(ring));
+            const uint32_t need = static_cast<uint32_t>(nvalid) * kChunkBytes;
+            if (off + need > static_cast<uint32_t>(ring)) {   // no room before the end: wrap
+                h += static_cast<uint32_t>(ring) - off;
+                off = 0;
+            }
+            const uint64_t h_end = h + need;
             int ok = 1;
-            if (lane == 0) ok = mbar_wait_bounded(&empty[s], ph ^ 1u) ? 1 : 0;
-            ok = __shfl_sync(kFullMask, ok, 0);
+            while (it - rel >= kRingEntries || h_end - tail > static_cast<uint64_t>(ring)) {
+                const int e = rel % kRingEntries;
+                if (lane == 0) ok = mbar_wait_bounded(&empty[e], static_cast<uint32_t>(rel / kRingEntries) & 1u) ? 1 : 0;
+                ok = __shfl_sync(kFullMask, ok, 0);
+                if (!ok) break;
+                tail = __shfl_sync(kFullMask, my_end, e);
+                ++rel;
+            }
             if (!ok) {
                 if (lane == 0) flag_error(err_flag, TK_DEVERR_TIMEOUT);
                 break;
             }
-            if (lane < k) {
-                meta[s].w[lane] = wl;
-                meta[s].valid[lane] = rowp != nullptr ? 1 : 0;
+            head = h_end;
+            const int e = it % kRingEntries;
+            if (lane == e) my_end = h_end;
+            if (rowp != nullptr) meta[e].w[pos] = wl;
+            if (lane == 0) {
+                meta[e].n = nvalid;
+                meta[e].off = off;
             }
-            const unsigned vmask = __ballot_sync(kFullMask, rowp != nullptr);
             __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(vmask)) * bytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[e], static_cast<uint32_t>(nvalid) * bytes);
             __syncwarp();
             if (rowp != nullptr) {
-                uint8_t* dst = data + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * kChunkBytes;
+                uint8_t* dst = data + off + static_cast<uint32_t>(pos) * kChunkBytes;
                 const uint8_t* src = rowp + static_cast<int64_t>(ch0) * 2;
-                if (TK_REDUCE_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, &full[s], l2_policy(TK_REDUCE_LOAD_POLICY));
-                else bulk_load(dst, src, bytes, &full[s]);
+                if (TK_REDUCE_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, &full[e], l2_policy(TK_REDUCE_LOAD_POLICY));
+                else bulk_load(dst, src, bytes, &full[e]);
             }
         }
     } else {
@@ -219,27 +241,27 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
         const int ct = threadIdx.x - 32;  // 0 .. 32*kConsumerWarps-1
         int it = 0;
         for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
-            const int s = it % S;
-            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-            if (!mbar_wait_bounded(&full[s], ph)) {
+            const int e = it % kRingEntries;
+            if (!mbar_wait_bounded(&full[e], static_cast<uint32_t>(it / kRingEntries) & 1u)) {
                 flag_error(err_flag, TK_DEVERR_TIMEOUT);
                 break;
             }
             const int64_t t = u / chunks;
             const int ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
             const int chn = min(kChunkCh, H - ch0);
+            const int n = meta[e].n;
+            const uint8_t* rows_at = data + meta[e].off;
 #pragma unroll
             for (int q = 0; q < kVecs; ++q) {
                 const int vec = ct + q * 32 * kConsumerWarps;   // 8-channel vector within the unit
                 if (vec * 8 >= chn) break;
                 float acc[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-                const uint8_t* base = data + static_cast<size_t>(s) * stage_bytes + vec * 16;
-                for (int j = 0; j < k; ++j) {
-                    if (!meta[s].valid[j]) continue;
-                    const float wj = meta[s].w[j];
-                    const uint4 q4 = *reinterpret_cast<const uint4*>(base + j * kChunkBytes);
+                for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+                const uint8_t* base = rows_at + vec * 16;
+                for (int i = 0; i < n; ++i) {   // the valid rows in slot order
+                    const float wj = meta[e].w[i];
+                    const uint4 q4 = *reinterpret_cast<const uint4*>(base + i * kChunkBytes);
                     acc[0] = __fmaf_rn(wj, lo_bf16(q4.x), acc[0]);
                     acc[1] = __fmaf_rn(wj, hi_bf16(q4.x), acc[1]);
                     acc[2] = __fmaf_rn(wj, lo_bf16(q4.y), acc[2]);
@@ -257,14 +279,14 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
                 st_v4(out + t * row_bytes + static_cast<int64_t>(ch0 + vec * 8) * 2, o);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&empty[e]);
         }
     }
 }
 
 struct LaunchShape {
-    int grid_cap = 0;   // SMs x resident CTAs for the current stage count
-    int S = 0;
+    int grid_cap = 0;   // SMs x resident CTAs for the current ring size
+    int ring = 0;       // ring bytes
 };
 
 // Launch shape for k on the current device, worked out once per row source (the kernel's
@@ -281,8 +303,8 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
     }
     std::lock_guard<std::mutex> lock(setup_mutex());
     if (!ready[dev][k].load(std::memory_order_relaxed)) {
-        const int S = stages_for(k);
-        const size_t smem = smem_bytes(k, S);
+        const int ring = ring_bytes_for(k);
+        const size_t smem = smem_bytes(ring);
         cudaError_t err = cudaSuccess;
         if (static_cast<int>(smem) > configured_smem[dev]) {
             err = cudaFuncSetAttribute(reduce_kernel<Rows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -294,7 +316,7 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
         err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows>, kRedThreads, smem);
         if (err != cudaSuccess) return err;
         shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
-        shapes[dev][k].S = S;
+        shapes[dev][k].ring = ring;
         ready[dev][k].store(true, std::memory_order_release);
     }
     out = shapes[dev][k];
@@ -312,8 +334,8 @@ cudaError_t launch_reduce(const Rows& rows, const float* w, int T, int k, int H,
     const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t units = static_cast<int64_t>(T) * chunks;
     const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);
-    return launch_pdl(reduce_kernel<Rows>, dim3(grid), dim3(kRedThreads), smem_bytes(k, shape.S),
-                      static_cast<cudaStream_t>(stream), rows, w, T, k, H, shape.S,
+    return launch_pdl(reduce_kernel<Rows>, dim3(grid), dim3(kRedThreads), smem_bytes(shape.ring),
+                      static_cast<cudaStream_t>(stream), rows, w, T, k, H, shape.ring,
                       static_cast<uint8_t*>(out), err_flag);
 }
 
