@@ -27,12 +27,23 @@ constexpr int kConsumerWarps = 4;
 constexpr int kBwdThreads = 32 * (1 + kConsumerWarps);
 constexpr int kChunkCh = 8 * 32 * kConsumerWarps;  // channels per unit, one vector per thread
 constexpr int kChunkBytes = kChunkCh * 2;
-constexpr int kStageBudget = 40 * 1024;
+#ifndef TK_BACKWARD_STAGE_KB
+#define TK_BACKWARD_STAGE_KB 40
+#endif
+#ifndef TK_BACKWARD_STORE_EVICT_FIRST   // d_y rows are written once and not read here
+#define TK_BACKWARD_STORE_EVICT_FIRST 1
+#endif
+constexpr int kStageBudget = TK_BACKWARD_STAGE_KB * 1024;
 constexpr int kRegRows = 8;  // up to this k, per-thread register accumulators for d_w
 
 #ifndef TK_BACKWARD_LOAD_POLICY   // L2 policy of the row loads: 0 none, 1 evict-normal, 2 evict-first
 #define TK_BACKWARD_LOAD_POLICY 1
 #endif
+
+__device__ __forceinline__ void store_dy(void* p, uint4 v) {
+    if (TK_BACKWARD_STORE_EVICT_FIRST) st_v4_hint(p, v, l2_policy_evict_first());
+    else st_v4(p, v);
+}
 
 __device__ __forceinline__ void load_row(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     if (TK_BACKWARD_LOAD_POLICY != 0) bulk_load_hint(dst, src, bytes, bar, l2_policy(TK_BACKWARD_LOAD_POLICY));
@@ -188,7 +199,7 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
                         o.y = pack_bf16x2(__fmul_rn(wj, gv[2]), __fmul_rn(wj, gv[3]));
                         o.z = pack_bf16x2(__fmul_rn(wj, gv[4]), __fmul_rn(wj, gv[5]));
                         o.w = pack_bf16x2(__fmul_rn(wj, gv[6]), __fmul_rn(wj, gv[7]));
-                        st_v4(dy_base + static_cast<int64_t>(sl) * row_bytes, o);
+                        store_dy(dy_base + static_cast<int64_t>(sl) * row_bytes, o);
                     }
                 } else {
                     for (int j = 0; j < k; ++j) {
@@ -208,7 +219,7 @@ reduce_backward_kernel(const uint8_t* __restrict__ g, const uint8_t* __restrict_
                             o.y = pack_bf16x2(__fmul_rn(wj, gv[2]), __fmul_rn(wj, gv[3]));
                             o.z = pack_bf16x2(__fmul_rn(wj, gv[4]), __fmul_rn(wj, gv[5]));
                             o.w = pack_bf16x2(__fmul_rn(wj, gv[6]), __fmul_rn(wj, gv[7]));
-                            st_v4(dy_base + static_cast<int64_t>(sl) * row_bytes, o);
+                            store_dy(dy_base + static_cast<int64_t>(sl) * row_bytes, o);
                         }
 #pragma unroll
                         for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(kFullMask, part, off);

@@ -210,4 +210,11 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                  : "memory");
 }
 
+// 16-byte store with an L2 cache-policy hint.
+__device__ __forceinline__ void st_v4_hint(void* p, uint4 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy)
+                 : "memory");
+}
+
 }  // namespace tk
