@@ -192,6 +192,23 @@ TK_API tk_status tk_balance_stats(const float* logits, const int32_t* counts, in
                                   size_t workspace_bytes, void* stream);
 
 /*
+ * The same statistics over a batch split across data-parallel ranks, in two calls around an
+ * all-reduce (the only exchange the routing path has):
+ *   tk_balance_score_sums: sums[e] = sum over this rank's T tokens of p[t,e] (double, the
+ *     per-64-token-tile partials added in tile order, as in tk_balance_stats);
+ *   tk_balance_finalize: from sums and counts summed over all ranks and the total token count
+ *     T_total: P = sums/T_total, f = E*counts/(k*T_total), loss = sum_e f*P (fixed-order tree).
+ * On one rank, tk_balance_score_sums then tk_balance_finalize(sums, counts, T) equals
+ * tk_balance_stats bit for bit.
+ *   sums      device, double [E];  workspace as for tk_balance_stats
+ */
+TK_API tk_status tk_balance_score_sums(const float* logits, int T, int E, int score_fn,
+                                       double* sums, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+TK_API tk_status tk_balance_finalize(const double* sums, const int32_t* counts, int64_t T_total,
+                                     int E, int k, float* P, float* f, float* loss, void* stream);
+
+/*
  * Tensor-parallel expert mask (147227.xyz "moe/": tensor-parallel mask; no definition on the
  * pages). Experts are owned in tp_size contiguous groups of E/tp_size; for rank tp_rank,
  * out_idx = topk_idx - tp_rank*E/tp_size where the expert is in the rank's group, else -1 (a

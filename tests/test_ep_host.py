@@ -73,3 +73,44 @@ def test_count_exchange_three_gloo_ranks(tmp_path, oracle_lib):
     world = 3
     mp.spawn(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
     assert (tmp_path / "ok").exists()
+
+
+def _balance_worker(rank, world, port, result_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as tdist
+
+    from token_routing_gate_b200 import dist
+
+    assert dist.init("gloo", timeout_s=60)
+    E = 16
+    g = torch.Generator().manual_seed(rank)
+    sums = torch.randint(0, 1 << 20, (E,), generator=g).to(torch.float64) / 64.0   # exact in double
+    counts = torch.randint(0, 1000, (E,), generator=g, dtype=torch.int32)
+    T = 100 + rank
+    s2, c2, T2 = dist.allreduce_balance_inputs(sums.clone(), counts, T)
+    gathered = [None] * world
+    tdist.all_gather_object(gathered, (sums, counts, T, s2, c2, T2))
+    if rank == 0:
+        want_s = sum(x[0] for x in gathered)
+        want_c = sum(x[1] for x in gathered)
+        for x in gathered:   # every rank holds the same totals
+            assert torch.equal(x[3], want_s) and torch.equal(x[4], want_c.to(torch.int32))
+            assert x[5] == sum(y[2] for y in gathered)
+        open(os.path.join(result_dir, "ok"), "w").close()
+    dist.finish()
+
+
+def test_balance_inputs_allreduce_three_gloo_ranks(tmp_path):
+    world = 3
+    mp.spawn(_balance_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    assert (tmp_path / "ok").exists()
+
+
+def test_balance_inputs_single_rank_unchanged():
+    from token_routing_gate_b200 import dist
+
+    sums = torch.arange(4, dtype=torch.float64)
+    counts = torch.arange(4, dtype=torch.int32)
+    s, c, T = dist.allreduce_balance_inputs(sums, counts, 7)
+    assert s is sums and c is counts and T == 7

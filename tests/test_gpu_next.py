@@ -38,6 +38,43 @@ def test_balance_stats_empty_batch():
     assert (P == 0).all() and (f == 0).all() and loss.item() == 0.0
 
 
+@pytest.mark.parametrize("wl", [W.MID, W.V3.with_(T=3000)], ids=lambda w: w.name)
+def test_balance_sums_then_finalize_is_the_one_call(wl):
+    logits, bias = W.gate_inputs(wl, "cuda")
+    idx, _ = tk.gate_topk(logits, wl.k, wl.score, bias)
+    rm = tk.route_map(idx, wl.E, 1)
+    one = tk.balance_stats(logits, rm.counts, wl.k, wl.score)
+    sums = tk.balance_score_sums(logits, wl.score)
+    two = tk.balance_finalize(sums, rm.counts, wl.T, wl.k)
+    torch.cuda.synchronize()
+    for a, b in zip(one, two):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("shards", [2, 3, 8])
+def test_global_balance_stats_over_rank_shards(shards):
+    # a batch split unevenly over ranks: per-rank sums and counts, added in rank order (what the
+    # all-reduce computes), then finalize == the statistics of the whole batch
+    wl = W.V3.with_(T=5000)
+    logits, bias = W.gate_inputs(wl, "cuda")
+    idx, _ = tk.gate_topk(logits, wl.k, wl.score, bias)
+    cuts = np.linspace(0, wl.T, shards + 1).astype(int)
+    cuts[1] = 7                                   # a tiny first shard
+    sums = torch.zeros(wl.E, dtype=torch.float64, device="cuda")
+    counts = torch.zeros(wl.E, dtype=torch.int32, device="cuda")
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        sums += tk.balance_score_sums(logits[a:b].contiguous(), wl.score)
+        counts += tk.route_map(idx[a:b].contiguous(), wl.E, 1).counts
+    P, f, loss = tk.balance_finalize(sums, counts, wl.T, wl.k)
+    full = tk.route_map(idx, wl.E, 1).counts
+    torch.cuda.synchronize()
+    assert torch.equal(counts, full)
+    Pr, fr, lr = oracle.balance_stats(logits.cpu().numpy(), full.cpu().numpy(), wl.k, oracle.SIGMOID)
+    np.testing.assert_allclose(P.cpu().numpy(), Pr, rtol=ULP32, atol=0)
+    np.testing.assert_allclose(f.cpu().numpy(), fr, rtol=ULP32, atol=0)
+    assert abs(loss.item() - lr) <= ULP32 * abs(lr)
+
+
 @pytest.mark.parametrize("tp", [1, 2, 8])
 def test_tp_mask_then_route(tp):
     wl = W.V3.with_(T=3000)

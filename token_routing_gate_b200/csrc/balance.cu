@@ -10,6 +10,9 @@
 //     its 8 warps in order and writes one row of a [tiles x E] partial-sum matrix.
 //   balance_final_kernel: one CTA sums each column in tile order, forms P, f and the loss with
 //     a fixed-order tree. The tiling depends on T only, so results do not depend on the GPU.
+// Over several data-parallel ranks the same statistics of the whole batch come from
+// tk_balance_score_sums (each rank's column sums, in tile order) + an all-reduce of the sums,
+// the counts and T + tk_balance_finalize (the final kernel over one "tile" of summed values).
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -99,7 +102,7 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
 
 __global__ void __launch_bounds__(kFinalThreads)
 balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_t* __restrict__ counts,
-                     int T, int E, int k, float* __restrict__ P, float* __restrict__ f,
+                     int64_t T, int E, int k, float* __restrict__ P, float* __restrict__ f,
                      float* __restrict__ loss) {
     __shared__ double prod[kFinalThreads];
     pdl_wait();
@@ -108,8 +111,8 @@ balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         double sum = 0.0;
         for (int c = 0; c < tiles; ++c) sum += partial[static_cast<int64_t>(c) * E + e];
-        const double Pe = T > 0 ? sum / T : 0.0;
-        const double fe = T > 0 ? static_cast<double>(E) * counts[e] / (static_cast<double>(k) * T) : 0.0;
+        const double Pe = T > 0 ? sum / static_cast<double>(T) : 0.0;
+        const double fe = T > 0 ? static_cast<double>(E) * counts[e] / (static_cast<double>(k) * static_cast<double>(T)) : 0.0;
         P[e] = static_cast<float>(Pe);
         f[e] = static_cast<float>(fe);
         mine += fe * Pe;
@@ -121,6 +124,17 @@ balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_
         __syncthreads();
     }
     if (threadIdx.x == 0) *loss = static_cast<float>(prod[0]);
+}
+
+// Column sums of the partial matrix in tile order (the same additions as the final kernel).
+__global__ void __launch_bounds__(kFinalThreads)
+balance_colsum_kernel(const double* __restrict__ partial, int tiles, int E, double* __restrict__ sums) {
+    pdl_wait();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        double sum = 0.0;
+        for (int c = 0; c < tiles; ++c) sum += partial[static_cast<int64_t>(c) * E + e];
+        sums[e] = sum;
+    }
 }
 
 template <int EPL>
@@ -152,6 +166,17 @@ __global__ void tp_mask_kernel(const int32_t* __restrict__ in, int64_t n, int lo
 }
 
 int stat_tiles(int T) { return (T + kStatTileTokens - 1) / kStatTileTokens; }
+
+cudaError_t launch_partials(const float* logits, int T, int E, int score_fn, double* partial,
+                            int tiles, cudaStream_t s) {
+    const int epl = (E + 31) / 32;
+    if (epl <= 1) return launch_partial<1>(logits, T, E, score_fn, partial, tiles, s);
+    if (epl <= 2) return launch_partial<2>(logits, T, E, score_fn, partial, tiles, s);
+    if (epl <= 4) return launch_partial<4>(logits, T, E, score_fn, partial, tiles, s);
+    if (epl <= 8) return launch_partial<8>(logits, T, E, score_fn, partial, tiles, s);
+    if (epl <= 16) return launch_partial<16>(logits, T, E, score_fn, partial, tiles, s);
+    return launch_partial<32>(logits, T, E, score_fn, partial, tiles, s);
+}
 
 }  // namespace
 }  // namespace tk
@@ -185,18 +210,57 @@ extern "C" tk_status tk_balance_stats(const float* logits, const int32_t* counts
     const int tiles = stat_tiles(T);
     cudaError_t err = cudaSuccess;
     if (tiles > 0) {
-        const int epl = (E + 31) / 32;
-        if (epl <= 1) err = launch_partial<1>(logits, T, E, score_fn, partial, tiles, s);
-        else if (epl <= 2) err = launch_partial<2>(logits, T, E, score_fn, partial, tiles, s);
-        else if (epl <= 4) err = launch_partial<4>(logits, T, E, score_fn, partial, tiles, s);
-        else if (epl <= 8) err = launch_partial<8>(logits, T, E, score_fn, partial, tiles, s);
-        else if (epl <= 16) err = launch_partial<16>(logits, T, E, score_fn, partial, tiles, s);
-        else err = launch_partial<32>(logits, T, E, score_fn, partial, tiles, s);
+        err = launch_partials(logits, T, E, score_fn, partial, tiles, s);
         if (err != cudaSuccess) return check_launch(err, "balance_partial_kernel");
     }
     err = launch_pdl(balance_final_kernel, dim3(1), dim3(kFinalThreads), 0, s,
-                     static_cast<const double*>(partial), tiles, counts, T, E, k, P, f, loss);
+                     static_cast<const double*>(partial), tiles, counts, static_cast<int64_t>(T), E,
+                     k, P, f, loss);
     return check_launch(err, "balance_final_kernel");
+}
+
+extern "C" tk_status tk_balance_score_sums(const float* logits, int T, int E, int score_fn,
+                                           double* sums, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_balance_score_sums: T=%d must be >= 0", T);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_balance_score_sums: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (score_fn != TK_SCORE_SOFTMAX && score_fn != TK_SCORE_SIGMOID)
+        return fail_arg("tk_balance_score_sums: unknown score_fn %d", score_fn);
+    if (sums == nullptr || workspace == nullptr)
+        return fail_arg("tk_balance_score_sums: sums and workspace must not be NULL");
+    if (T > 0 && logits == nullptr) return fail_arg("tk_balance_score_sums: logits must not be NULL");
+    const size_t need = tk_balance_stats_workspace_bytes(T, E);
+    if (workspace_bytes < need)
+        return fail_arg("tk_balance_score_sums: workspace holds %zu bytes, needs %zu", workspace_bytes, need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+        return fail_arg("tk_balance_score_sums: workspace must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    double* partial = static_cast<double*>(workspace);
+    const int tiles = stat_tiles(T);
+    if (tiles > 0) {
+        const cudaError_t e = launch_partials(logits, T, E, score_fn, partial, tiles, s);
+        if (e != cudaSuccess) return check_launch(e, "balance_partial_kernel");
+    }
+    const cudaError_t e = launch_pdl(balance_colsum_kernel, dim3(1), dim3(kFinalThreads), 0, s,
+                                     static_cast<const double*>(partial), tiles, E, sums);
+    return check_launch(e, "balance_colsum_kernel");
+}
+
+extern "C" tk_status tk_balance_finalize(const double* sums, const int32_t* counts, int64_t T,
+                                         int E, int k, float* P, float* f, float* loss,
+                                         void* stream) {
+    using namespace tk;
+    if (T < 0) return fail_arg("tk_balance_finalize: T=%lld must be >= 0", (long long)T);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_balance_finalize: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
+    if (k < 1 || k > E || k > TK_MAX_TOPK)
+        return fail_arg("tk_balance_finalize: k=%d outside [1, min(E=%d, %d)]", k, E, TK_MAX_TOPK);
+    if (sums == nullptr || counts == nullptr || P == nullptr || f == nullptr || loss == nullptr)
+        return fail_arg("tk_balance_finalize: sums, counts, P, f and loss must not be NULL");
+    const cudaError_t e = launch_pdl(balance_final_kernel, dim3(1), dim3(kFinalThreads), 0,
+                                     static_cast<cudaStream_t>(stream), sums, 1, counts, T, E, k, P,
+                                     f, loss);
+    return check_launch(e, "balance_final_kernel");
 }
 
 extern "C" tk_status tk_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size,

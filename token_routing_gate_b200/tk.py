@@ -26,7 +26,7 @@ DEVERR_TIMEOUT = 16
 # every C entry point declared in include/tk_route.h
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
                "tk_route_map_static", "tk_expand", "tk_reduce", "tk_balance_stats_workspace_bytes",
-               "tk_balance_stats", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
+               "tk_balance_stats", "tk_balance_score_sums", "tk_balance_finalize", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
                "tk_reduce_backward", "tk_expand_backward", "tk_ep_layout_workspace_bytes",
                "tk_ep_layout", "tk_ep_dispatch", "tk_ep_combine", "tk_selftest_bounded_wait",
                "tk_status_str", "tk_last_error_detail", "tk_abi_version")
@@ -70,6 +70,10 @@ def _load():
     L.tk_balance_stats_workspace_bytes.restype = sz
     L.tk_balance_stats.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
     L.tk_balance_stats.restype = i32
+    L.tk_balance_score_sums.argtypes = [vp, i32, i32, i32, vp, vp, sz, vp]
+    L.tk_balance_score_sums.restype = i32
+    L.tk_balance_finalize.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp]
+    L.tk_balance_finalize.restype = i32
     L.tk_tp_mask.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp]
     L.tk_tp_mask.restype = i32
     L.tk_reduce_backward_workspace_bytes.argtypes = [i32, i32]
@@ -214,6 +218,32 @@ def balance_stats(logits, counts, k, score="sigmoid", workspace=None, out=None, 
     _check("tk_balance_stats", lib.tk_balance_stats(
         _ptr(logits), _ptr(counts), T, E, k, SCORE[score], _ptr(P), _ptr(f), _ptr(loss),
         _ptr(workspace), workspace.numel(), _stream(stream)))
+    return P, f, loss
+
+
+def balance_score_sums(logits, score="sigmoid", workspace=None, out=None, stream=None):
+    """Per-expert sums (double [E]) of the normalised unbiased scores over this batch's tokens."""
+    T, E = logits.shape
+    dev = logits.device
+    if workspace is None:
+        workspace = _workspace(int(lib.tk_balance_stats_workspace_bytes(T, E)), dev)
+    if out is None:
+        out = torch.empty(E, dtype=torch.float64, device=dev)
+    _check("tk_balance_score_sums", lib.tk_balance_score_sums(
+        _ptr(logits), T, E, SCORE[score], _ptr(out), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out
+
+
+def balance_finalize(sums, counts, T_total, k, out=None, stream=None):
+    """(P, f, loss) fp32 from score sums and counts summed over ranks and the total token count."""
+    E = sums.shape[0]
+    dev = sums.device
+    if out is None:
+        out = (torch.empty(E, device=dev), torch.empty(E, device=dev), torch.empty(1, device=dev))
+    P, f, loss = out
+    _check("tk_balance_finalize", lib.tk_balance_finalize(
+        _ptr(sums), _ptr(counts), int(T_total), E, k, _ptr(P), _ptr(f), _ptr(loss), _stream(stream)))
     return P, f, loss
 
 
