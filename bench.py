@@ -4,7 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tk|reference] [--workload NAME]
 
 One step = the four C-ABI calls (tk_gate_topk, tk_route_map, tk_expand, tk_reduce) over one
-synthetic batch, inputs resident in HBM. Prints ONE JSON line (rank 0). For N > 1 run it under
+synthetic batch, inputs resident in HBM. The headline runs K such steps with two batches in
+flight (the next batch's gate + route map on a second stream while this batch's expand + reduce
+run); the JSON line also carries the serial time of the same K steps. Prints ONE JSON line (rank 0). For N > 1 run it under
 torchrun: every rank routes its own batch (weak scaling, no data-path collective), time is the
 max over ranks.
 
@@ -326,20 +328,41 @@ def run_tk(args, wl):
     R = int(rm.offsets[-1].item())
 
     K = args.steps
-    # Pass 1 (the headline): K steps with nothing between the calls, so each kernel's launch
-    # overlaps the end of the previous one as it would in a model.
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier(dev_for_collectives)
+    from token_routing_gate_b200.pipeline import RoutingPipeline
+
+    pipe = RoutingPipeline(wl.T, wl.E, wl.k, wl.score, wl.align, device=dev)
+
+    def pipelined(n):
+        """n batches, two in flight: batch i+1's gate + route map on the pipeline's stream while
+        batch i's expand + reduce run on `stream`."""
+        pipe.stream.wait_stream(stream)
+        h = pipe.route(logits, bias)
+        for i in range(n):
+            nxt = pipe.route(logits, bias) if i + 1 < n else None
+            pipe.dispatch_combine(h, x, y, out, xe, wl.out_dtype, xs, stream=stream)
+            h = nxt
+
+    for _ in range(args.warmup):
+        pipelined(2)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clocks:
+
+    def timed(run):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier(dev_for_collectives)
+        torch.cuda.synchronize(dev)
         start.record(stream)
-        for i in range(K):
-            step()
+        run()
         end.record(stream)
         torch.cuda.synchronize(dev)
-    dist.barrier(dev_for_collectives)
-    elapsed_s = start.elapsed_time(end) / 1e3
-    max_s = dist.max_over_ranks(elapsed_s, dev_for_collectives)
+        dist.barrier(dev_for_collectives)
+        return dist.max_over_ranks(start.elapsed_time(end) / 1e3, dev_for_collectives)
+
+    # Pass 1 (the headline): K batches with two in flight (RoutingPipeline), nothing between the
+    # calls, so each kernel's launch also overlaps the end of the previous one.
+    with ClockSampler(dev.index) as clocks:
+        max_s = timed(lambda: pipelined(K))
+    # Pass 1b: the same K steps one after another on one stream (no batch overlap).
+    serial_s = timed(lambda: [step() for _ in range(K)])
     # Pass 2 (the per-kernel breakdown behind the roofline): the same K steps with events
     # between the calls; the events stop one call's launch from overlapping the previous one.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
@@ -366,13 +389,19 @@ def run_tk(args, wl):
     line = {
         "metric": METRIC, "value": dist.aggregate_rate(wl.T * K, world, max_s), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * max_s / K,
+        "serial": {"value": dist.aggregate_rate(wl.T * K, world, serial_s),
+                   "ms_per_step": 1e3 * serial_s / K,
+                   "note": "the same K steps one after another on one stream"},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "E": wl.E, "k": wl.k, "H": wl.H,
                    "score": wl.score, "bias": wl.bias, "align": wl.align,
                    "out_dtype": wl.out_dtype, "tokens_per_rank": wl.T, "rows_used": R,
                    "l2": "no flush: each step touches %.2f GB (> 126 MB L2)" % (sum(ab.values()) / 1e9),
-                   "parallelism": f"dp{world} (independent token shards, no data-path collective)"},
+                   "parallelism": f"dp{world} (independent token shards, no data-path collective)",
+                   "pipelining": "two batches in flight: gate + route map of batch i+1 on a second "
+                                 "stream overlap expand + reduce of batch i (RoutingPipeline); "
+                                 "every batch runs all four calls"},
         "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": ncu_traffic(dom_file, dom_kernel, wl.name),
