@@ -174,6 +174,18 @@ TK_API tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slot_of
                     int k, int H, void* out, int32_t* err_flag, void* stream);
 
 /*
+ * tk_reduce for slot maps in which most pairs are masked (-1): the rows an expert-parallel
+ * destination receives (each lists k choices, about k/G of them local) or a route map after
+ * tk_tp_mask. Same arguments, arithmetic and results, bit for bit. It steps through its work
+ * units with O(1) updates instead of a 64-bit division per unit, which is what limits units with
+ * few valid rows (measured on B200: the reduce of an expert-parallel destination 22 % faster);
+ * with every pair valid tk_reduce is the faster of the two (by about 2 %).
+ */
+TK_API tk_status tk_reduce_masked(const void* y, int64_t y_rows, const int32_t* slot_of,
+                                  const float* w, int T, int k, int H, void* out,
+                                  int32_t* err_flag, void* stream);
+
+/*
  * Load-balance statistics (147227.xyz "moe/": load-balance loss computation; no formula on the
  * pages -- this is the usual auxiliary balance loss of routed MoE layers). With p[t,i] the
  * unbiased scores of token t normalised over all E experts (softmax, or sigmoid divided by its

@@ -132,6 +132,21 @@ def test_reduce_rejects(tk):
     assert L.tk_reduce(None, 0, None, None, 0, 2, 256, None, None, None) == 0
 
 
+def test_reduce_masked_validates_like_reduce(tk):
+    L = tk.lib
+    ok = [FAKE, 10, FAKE, None, 4, 2, 256, FAKE, None, None]
+    for i, v, what in [(5, 0, "k"), (5, 33, "k"), (6, 12, "H"), (1, -1, "y_rows"), (2, None, "NULL"),
+                       (7, MISALIGNED, "aligned")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_reduce_masked(*a) == 1, what
+        detail = L.tk_last_error_detail().decode()
+        assert what in detail and "tk_reduce_masked" in detail
+    a = list(ok)
+    a[4] = 0
+    assert L.tk_reduce_masked(*a) == 0      # T = 0: nothing to do
+
+
 def test_binding_raises_with_detail(tk):
     with pytest.raises(tk.TkError) as ei:
         tk._check("tk_reduce", tk.lib.tk_reduce(FAKE, 1, FAKE, None, 4, 0, 256, FAKE, None, None))

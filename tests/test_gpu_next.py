@@ -75,6 +75,35 @@ def test_global_balance_stats_over_rank_shards(shards):
     assert abs(loss.item() - lr) <= ULP32 * abs(lr)
 
 
+@pytest.mark.parametrize("case", ["dense", "tp8", "ep_like", "ragged"])
+def test_reduce_masked_equals_reduce(case):
+    wl = {"dense": W.V3.with_(T=3000, H=1024), "tp8": W.V3.with_(T=4000, H=512),
+          "ep_like": W.V3.with_(T=2500, H=7168), "ragged": W.MID.with_(T=777, H=200)}[case]
+    logits, bias = W.gate_inputs(wl, "cuda")
+    idx, w = tk.gate_topk(logits, wl.k, wl.score, bias)
+    E = wl.E
+    if case == "tp8":                       # 7/8 of the pairs masked
+        idx = tk.tp_mask(idx, wl.E, 8, 3)
+        E = wl.E // 8
+    if case == "ep_like":                   # keep one expert group of eight, as a destination would
+        idx = torch.where((idx // 32) == 5, idx - 160, torch.full_like(idx, -1))
+        E = 32
+    rm = tk.route_map(idx, E, 1)
+    y = W.expert_outputs(wl.with_(E=E), "cuda", rows=max(tk.max_rows(wl.T, E, wl.k, 1), 1))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    a = tk.reduce(y, rm.slot_of, w, err_flag=err)
+    b = tk.reduce(y, rm.slot_of, w, err_flag=err, masked=True)
+    c = tk.reduce(y, rm.slot_of, None, err_flag=err, masked=True)
+    d = tk.reduce(y, rm.slot_of, None, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(c.view(torch.int16), d.view(torch.int16))
+    if case == "ragged":                    # and the oracle, element by element
+        ref = oracle.reduce(bf16_bits(y), rm.slot_of.cpu().numpy(), w.cpu().numpy())
+        assert bf16_ulp_diff(bf16_bits(b), ref).max() <= 1
+
+
 @pytest.mark.parametrize("tp", [1, 2, 8])
 def test_tp_mask_then_route(tp):
     wl = W.V3.with_(T=3000)

@@ -138,7 +138,9 @@ struct RankRows {
     }
 };
 
-template <class Rows>
+// kStep: step each unit's (token, chunk) and ring offset by O(1) updates instead of 64-bit
+// division and modulo (the tk_reduce_masked form; see the entry points).
+template <class Rows, bool kStep>
 __global__ void __launch_bounds__(kRedThreads)
 reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, int T, int k, int H,
               int ring, uint8_t* __restrict__ out, int32_t* err_flag) {
@@ -162,6 +164,12 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
     const int chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t units = static_cast<int64_t>(T) * chunks;
     const int64_t row_bytes = static_cast<int64_t>(H) * 2;
+    // kStep: a CTA's units are blockIdx.x, blockIdx.x + G, ... (G = gridDim.x); unit u is token
+    // u / chunks, chunk u % chunks, both stepped by (G / chunks, G % chunks).
+    const int64_t step_t = static_cast<int64_t>(gridDim.x) / chunks;
+    const int step_c = static_cast<int>(static_cast<int64_t>(gridDim.x) - step_t * chunks);
+    const int64_t t_first = static_cast<int64_t>(blockIdx.x) / chunks;
+    const int c_first = static_cast<int>(static_cast<int64_t>(blockIdx.x) - t_first * chunks);
 
     if (warp == 0) {
         // ---------------- producer. Unit `it` takes entry it % kRingEntries and the next
@@ -181,24 +189,50 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
         uint64_t head = 0, tail = 0;   // ring bytes handed out / released so far
         uint64_t my_end = 0;           // lane e: end of entry e's bytes
         int rel = 0;                   // units known to be released
+        int64_t st_tn = t_first + step_t;   // kStep: token of the next unit, this unit's chunk,
+        int st_cn = c_first + step_c;       // the next unit's chunk, the ring offset
+        if (st_cn >= chunks) {
+            st_cn -= chunks;
+            ++st_tn;
+        }
+        int st_c = c_first;
+        uint32_t ring_off = 0;
         for (int it = 0; u < units; u += gridDim.x, ++it) {
-            const int64_t t = u / chunks;
-            const int ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
+            int ch0;
+            if constexpr (kStep) {
+                ch0 = st_c * kChunkCh;
+            } else {
+                const int64_t t = u / chunks;
+                ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
+            }
             const uint32_t bytes = static_cast<uint32_t>(min(kChunkCh, H - ch0)) * 2u;
             const int64_t raw = nxt_sl;
             const float wl = nxt_w;
             const int64_t un = u + gridDim.x;
             if (lane < k && un < units) {
-                const int64_t tn = un / chunks;
+                int64_t tn;
+                if constexpr (kStep) tn = st_tn;
+                else tn = un / chunks;
                 nxt_sl = rows.fetch(tn, lane, k);
                 if (w != nullptr) nxt_w = w[tn * k + lane];
+            }
+            if constexpr (kStep) {
+                st_c = st_cn;
+                st_tn += step_t;
+                st_cn += step_c;
+                if (st_cn >= chunks) {
+                    st_cn -= chunks;
+                    ++st_tn;
+                }
             }
             const uint8_t* rowp = lane < k ? rows.resolve(lctx, raw, row_bytes, err_flag) : nullptr;
             const unsigned vmask = __ballot_sync(kFullMask, rowp != nullptr);
             const int nvalid = __popc(vmask);
             const int pos = __popc(vmask & ((1u << lane) - 1u));   // this row's place among them
             uint64_t h = head;
-            uint32_t off = static_cast<uint32_t>(h % static_cast<uint64_t>(ring));
+            uint32_t off;
+            if constexpr (kStep) off = ring_off;
+            else off = static_cast<uint32_t>(h % static_cast<uint64_t>(ring));
             const uint32_t need = static_cast<uint32_t>(nvalid) * kChunkBytes;
             if (off + need > static_cast<uint32_t>(ring)) {   // no room before the end: wrap
                 h += static_cast<uint32_t>(ring) - off;
@@ -219,6 +253,7 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
                 break;
             }
             head = h_end;
+            if constexpr (kStep) ring_off = off + need;
             const int e = it % kRingEntries;
             if (lane == e) my_end = h_end;
             if (rowp != nullptr) meta[e].w[pos] = wl;
@@ -240,14 +275,29 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
         // ---------------- consumers
         const int ct = threadIdx.x - 32;  // 0 .. 32*kConsumerWarps-1
         int it = 0;
+        int64_t st_t = t_first;   // kStep: this unit's token and chunk
+        int st_c = c_first;
         for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
             const int e = it % kRingEntries;
             if (!mbar_wait_bounded(&full[e], static_cast<uint32_t>(it / kRingEntries) & 1u)) {
                 flag_error(err_flag, TK_DEVERR_TIMEOUT);
                 break;
             }
-            const int64_t t = u / chunks;
-            const int ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
+            int64_t t;
+            int ch0;
+            if constexpr (kStep) {
+                t = st_t;
+                ch0 = st_c * kChunkCh;
+                st_t += step_t;
+                st_c += step_c;
+                if (st_c >= chunks) {
+                    st_c -= chunks;
+                    ++st_t;
+                }
+            } else {
+                t = u / chunks;
+                ch0 = static_cast<int>(u - t * chunks) * kChunkCh;
+            }
             const int chn = min(kChunkCh, H - ch0);
             const int n = meta[e].n;
             const uint8_t* rows_at = data + meta[e].off;
@@ -291,7 +341,7 @@ struct LaunchShape {
 
 // Launch shape for k on the current device, worked out once per row source (the kernel's
 // shared-memory limit is raised to the largest size any k needs).
-template <class Rows>
+template <class Rows, bool kStep>
 cudaError_t launch_shape(int k, LaunchShape& out) {
     static LaunchShape shapes[kMaxDevices][TK_MAX_TOPK + 1];
     static std::atomic<bool> ready[kMaxDevices][TK_MAX_TOPK + 1];
@@ -307,13 +357,13 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
         const size_t smem = smem_bytes(ring);
         cudaError_t err = cudaSuccess;
         if (static_cast<int>(smem) > configured_smem[dev]) {
-            err = cudaFuncSetAttribute(reduce_kernel<Rows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(reduce_kernel<Rows, kStep>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
             if (err != cudaSuccess) return err;
             configured_smem[dev] = static_cast<int>(smem);
         }
         int per_sm = 0;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows>, kRedThreads, smem);
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows, kStep>, kRedThreads, smem);
         if (err != cudaSuccess) return err;
         shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
         shapes[dev][k].ring = ring;
@@ -323,18 +373,18 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
     return cudaSuccess;
 }
 
-template <class Rows>
+template <class Rows, bool kStep = false>
 cudaError_t launch_reduce(const Rows& rows, const float* w, int T, int k, int H, void* out,
                           int32_t* err_flag, void* stream, const char** what) {
     *what = "reduce_kernel setup";
     LaunchShape shape;
-    const cudaError_t e = launch_shape<Rows>(k, shape);
+    const cudaError_t e = launch_shape<Rows, kStep>(k, shape);
     if (e != cudaSuccess) return e;
     *what = "reduce_kernel";
     const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t units = static_cast<int64_t>(T) * chunks;
     const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);
-    return launch_pdl(reduce_kernel<Rows>, dim3(grid), dim3(kRedThreads), smem_bytes(shape.ring),
+    return launch_pdl(reduce_kernel<Rows, kStep>, dim3(grid), dim3(kRedThreads), smem_bytes(shape.ring),
                       static_cast<cudaStream_t>(stream), rows, w, T, k, H, shape.ring,
                       static_cast<uint8_t*>(out), err_flag);
 }
@@ -342,22 +392,41 @@ cudaError_t launch_reduce(const Rows& rows, const float* w, int T, int k, int H,
 }  // namespace
 }  // namespace tk
 
-extern "C" tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slot_of, const float* w,
-                               int T, int k, int H, void* out, int32_t* err_flag, void* stream) {
-    using namespace tk;
-    if (T < 0) return fail_arg("tk_reduce: T=%d must be >= 0", T);
-    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("tk_reduce: k=%d outside [1, %d]", k, TK_MAX_TOPK);
-    if (H < 8 || H % 8 != 0) return fail_arg("tk_reduce: H=%d must be a positive multiple of 8", H);
-    if (y_rows < 0) return fail_arg("tk_reduce: y_rows=%lld must be >= 0", (long long)y_rows);
+namespace tk {
+namespace {
+
+template <bool kStep>
+tk_status reduce_entry(const char* name, const void* y, int64_t y_rows, const int32_t* slot_of,
+                       const float* w, int T, int k, int H, void* out, int32_t* err_flag,
+                       void* stream) {
+    if (T < 0) return fail_arg("%s: T=%d must be >= 0", name, T);
+    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("%s: k=%d outside [1, %d]", name, k, TK_MAX_TOPK);
+    if (H < 8 || H % 8 != 0) return fail_arg("%s: H=%d must be a positive multiple of 8", name, H);
+    if (y_rows < 0) return fail_arg("%s: y_rows=%lld must be >= 0", name, (long long)y_rows);
     if (T == 0) return TK_OK;
     if (slot_of == nullptr || out == nullptr || (y == nullptr && y_rows > 0))
-        return fail_arg("tk_reduce: y, slot_of and out must not be NULL");
+        return fail_arg("%s: y, slot_of and out must not be NULL", name);
     if (reinterpret_cast<uintptr_t>(y) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 16 != 0)
-        return fail_arg("tk_reduce: y and out must be 16-byte aligned");
+        return fail_arg("%s: y and out must be 16-byte aligned", name);
     const SlotRows rows{static_cast<const uint8_t*>(y), y_rows, slot_of};
     const char* what = "";
-    const cudaError_t err = launch_reduce(rows, w, T, k, H, out, err_flag, stream, &what);
+    const cudaError_t err = launch_reduce<SlotRows, kStep>(rows, w, T, k, H, out, err_flag, stream, &what);
     return check_launch(err, what);
+}
+
+}  // namespace
+}  // namespace tk
+
+extern "C" tk_status tk_reduce(const void* y, int64_t y_rows, const int32_t* slot_of, const float* w,
+                               int T, int k, int H, void* out, int32_t* err_flag, void* stream) {
+    return tk::reduce_entry<false>("tk_reduce", y, y_rows, slot_of, w, T, k, H, out, err_flag, stream);
+}
+
+extern "C" tk_status tk_reduce_masked(const void* y, int64_t y_rows, const int32_t* slot_of,
+                                      const float* w, int T, int k, int H, void* out,
+                                      int32_t* err_flag, void* stream) {
+    return tk::reduce_entry<true>("tk_reduce_masked", y, y_rows, slot_of, w, T, k, H, out, err_flag,
+                                  stream);
 }
 
 extern "C" tk_status tk_ep_combine(const void* const* partial, const int64_t* base_row,

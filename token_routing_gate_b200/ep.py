@@ -80,7 +80,7 @@ def local_combine(bufs, n, E_local, align, expert_fn, d, stream=None):
         return None
     rm = tk.route_map(bufs.idx[:n], E_local, align, stream=stream)
     y = expert_fn(d, bufs, n, rm)
-    tk.reduce(y, rm.slot_of, bufs.w[:n], out=bufs.partial[:n], stream=stream)
+    tk.reduce(y, rm.slot_of, bufs.w[:n], out=bufs.partial[:n], stream=stream, masked=True)
     return rm
 
 

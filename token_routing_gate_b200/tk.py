@@ -25,7 +25,7 @@ DEVERR_TIMEOUT = 16
 
 # every C entry point declared in include/tk_route.h
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
-               "tk_route_map_static", "tk_expand", "tk_reduce", "tk_balance_stats_workspace_bytes",
+               "tk_route_map_static", "tk_expand", "tk_reduce", "tk_reduce_masked", "tk_balance_stats_workspace_bytes",
                "tk_balance_stats", "tk_balance_score_sums", "tk_balance_finalize", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
                "tk_reduce_backward", "tk_expand_backward", "tk_ep_layout_workspace_bytes",
                "tk_ep_layout", "tk_ep_dispatch", "tk_ep_combine", "tk_selftest_bounded_wait",
@@ -66,6 +66,8 @@ def _load():
     L.tk_expand.restype = i32
     L.tk_reduce.argtypes = [vp, i64, vp, vp, i32, i32, i32, vp, vp, vp]
     L.tk_reduce.restype = i32
+    L.tk_reduce_masked.argtypes = L.tk_reduce.argtypes
+    L.tk_reduce_masked.restype = i32
     L.tk_balance_stats_workspace_bytes.argtypes = [i32, i32]
     L.tk_balance_stats_workspace_bytes.restype = sz
     L.tk_balance_stats.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
@@ -189,14 +191,16 @@ def expand(x, rm, E, k, out_dtype="bf16", out=None, out_scale=None, err_flag=Non
     return (out, out_scale) if out_dtype == "fp8" else out
 
 
-def reduce(y, slot_of, w=None, out=None, err_flag=None, stream=None):
-    """y bf16 [rows,H], slot_of int32 [T,k], w fp32 [T,k] or None -> out bf16 [T,H]."""
+def reduce(y, slot_of, w=None, out=None, err_flag=None, stream=None, masked=False):
+    """y bf16 [rows,H], slot_of int32 [T,k], w fp32 [T,k] or None -> out bf16 [T,H].
+    masked=True calls tk_reduce_masked (same results; faster when most pairs are -1)."""
     T, k = slot_of.shape
     H = y.shape[1]
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device)
-    _check("tk_reduce", lib.tk_reduce(_ptr(y), y.shape[0], _ptr(slot_of), _ptr(w), T, k, H,
-                                      _ptr(out), _ptr(err_flag), _stream(stream)))
+    fn, name = (lib.tk_reduce_masked, "tk_reduce_masked") if masked else (lib.tk_reduce, "tk_reduce")
+    _check(name, fn(_ptr(y), y.shape[0], _ptr(slot_of), _ptr(w), T, k, H, _ptr(out), _ptr(err_flag),
+                    _stream(stream)))
     return out
 
 
