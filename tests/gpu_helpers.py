@@ -28,7 +28,7 @@ def score_fn(wl):
     return oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
 
 
-class GpuRun:
+class DeviceRun:
     """The four C-ABI calls on device tensors, with an error flag."""
 
     def __init__(self, wl, logits, bias, x, y, renormalize=True, stream=None):

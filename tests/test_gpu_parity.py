@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import GpuRun, assert_weights_close, bf16_bits, bf16_ulp_diff, score_fn
+from gpu_helpers import DeviceRun, assert_weights_close, bf16_bits, bf16_ulp_diff, score_fn
 from token_routing_gate_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -45,7 +45,7 @@ def test_small_workload_full_parity(wl):
     torch.manual_seed(0)
     logits, bias, x, y = _inputs(wl, "cpu")
     dev = [t.cuda() if t is not None else None for t in (logits, bias, x, y)]
-    run = GpuRun(wl, *dev)
+    run = DeviceRun(wl, *dev)
     assert run.err.item() == 0
     o_idx, o_w, slot_of, offsets = _check_gate_and_route(wl, run, logits, bias)
     R = int(offsets[-1])
@@ -62,7 +62,7 @@ def test_small_workload_full_parity(wl):
 @pytest.mark.parametrize("wl", LARGE, ids=lambda w: w.name)
 def test_large_workload_parity(wl):
     logits, bias, x, y = _inputs(wl, "cuda")
-    run = GpuRun(wl, logits, bias, x, y)
+    run = DeviceRun(wl, logits, bias, x, y)
     assert run.err.item() == 0
     o_idx, o_w, slot_of, offsets = _check_gate_and_route(wl, run, logits, bias)
     R = int(offsets[-1])
@@ -102,8 +102,8 @@ def test_large_workload_parity(wl):
 def test_pipeline_is_deterministic():
     wl = W.V3_FP8.with_(T=2048)
     logits, bias, x, y = _inputs(wl, "cuda")
-    a = GpuRun(wl, logits, bias, x, y)
-    b = GpuRun(wl, logits, bias, x, y)
+    a = DeviceRun(wl, logits, bias, x, y)
+    b = DeviceRun(wl, logits, bias, x, y)
     for name in ("idx", "w", "xq", "xs", "out"):
         assert torch.equal(getattr(a, name).view(torch.uint8), getattr(b, name).view(torch.uint8)), name
     for name in ("counts", "offsets", "slot_of", "token_of"):
@@ -136,7 +136,7 @@ def test_random_shapes_against_oracle(case):
                     out_dtype, _BASE + 1000 + case)
     logits, b, x, y = _inputs(wl, "cpu")
     dev = [t.cuda() if t is not None else None for t in (logits, b, x, y)]
-    run = GpuRun(wl, *dev)
+    run = DeviceRun(wl, *dev)
     assert run.err.item() == 0
     o_idx, o_w, slot_of, offsets = _check_gate_and_route(wl, run, logits, b)
     R = int(offsets[-1])
