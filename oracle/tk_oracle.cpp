@@ -531,8 +531,13 @@ int tko_ep_recv_bases(const int32_t* count_matrix, int G, int64_t* base, int64_t
     for (int d = 0; d < G; ++d) {
         int64_t acc = 0;
         for (int s = 0; s < G; ++s) {
+#if TKO_PLANT == 16
+            acc += count_matrix[static_cast<int64_t>(s) * G + d];  /* planted: inclusive prefix */
+            base[static_cast<int64_t>(s) * G + d] = acc;
+#else
             base[static_cast<int64_t>(s) * G + d] = acc;
             acc += count_matrix[static_cast<int64_t>(s) * G + d];
+#endif
         }
         recv_rows[d] = acc;
     }

@@ -2,7 +2,8 @@
 tie-break, biased weights, an off-by-one padding, unstable slots, the wrong E4M3 rounding or
 scale, the wrong reduction order, truncating bf16 rounding, a missing factor in the balance
 loss, a weighted gradient, an un-renumbered TP mask, the expert-parallel combine in the wrong
-rank order, experts dealt round-robin over ranks, global expert ids sent) is compiled into a copy of the oracle,
+rank order, experts dealt round-robin over ranks, global expert ids sent, inclusive receive
+bases) is compiled into a copy of the oracle,
 and the pins that cover that step must fail against it. The unplanted build must pass them."""
 import os
 import subprocess
@@ -30,6 +31,7 @@ MUTATIONS = {
     13: "ep_combine_rank_order",
     14: "ep_layout or ep_dispatch",
     15: "ep_dispatch",
+    16: "ep_recv_bases or ep_hand_case",
 }
 
 

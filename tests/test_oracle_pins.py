@@ -676,3 +676,28 @@ def test_ep_closed_form_equal_rows(oracle_lib):
     r = oracle_lib.ep_forward(xs, idxs, ws, lambda d, n: np.tile(v, (n, 1)), E, G)
     for s in range(G):
         assert np.all(r["out"][s] == v[None, :])
+
+
+@pytest.mark.parametrize("case", HAND["ep"], ids=lambda c: c["name"])
+def test_ep_hand_case(oracle_lib, case):
+    E, G, H = case["E"], case["G"], case["H"]
+    idxs = [np.array(s["idx"], dtype=np.int32) for s in case["sources"]]
+    ws = [np.array(s["w"], dtype=np.float32) for s in case["sources"]]
+    xs = [_bf16_bits(np.full((len(s["idx"]), H), 1.0)) for s in case["sources"]]
+    ys = [np.asarray(r, dtype=np.float64) for r in case["y_rows"]]
+
+    def make_y(d, rows):
+        y = np.zeros((rows, H))
+        y[:len(ys[d])] = ys[d][:, None]
+        return _bf16_bits(y)
+
+    r = oracle_lib.ep_forward(xs, idxs, ws, make_y, E, G)
+    assert r["count_matrix"].tolist() == case["send_counts"]
+    assert [lay[1].tolist() for lay in r["layout"]] == case["dest_pos"]
+    assert r["base"].tolist() == case["base"] and r["recv_rows"].tolist() == case["recv_rows"]
+    for d in range(G):
+        assert r["recv"][d][2].tolist() == case["recv_idx"][d]
+        assert r["recv"][d][3].tolist() == case["recv_w"][d]
+        assert r["dest"][d]["offsets"].tolist() == case["dest_offsets"][d]
+    for s, want in enumerate(case["out"]):
+        np.testing.assert_array_equal(r["out"][s], _bf16_bits(np.repeat(np.array(want)[:, None], H, 1)))
