@@ -114,3 +114,41 @@ def test_balance_inputs_single_rank_unchanged():
     counts = torch.arange(4, dtype=torch.int32)
     s, c, T = dist.allreduce_balance_inputs(sums, counts, 7)
     assert s is sums and c is counts and T == 7
+
+
+def test_epgroup_carves_one_symmetric_allocation(monkeypatch):
+    # EpGroup's host logic with torch's symmetric memory replaced by a CPU fake: every field of
+    # the receive buffers is a view of the one allocation at the offset that the peer addresses
+    # use, fields are 256-byte aligned and do not overlap, and each rank's addresses are its base
+    # plus the same offsets
+    import torch.distributed as tdist
+    import torch.distributed._symmetric_memory as symm
+
+    from token_routing_gate_b200 import ep
+
+    class FakeHandle:
+        def __init__(self, t):
+            self.buffer_ptrs = [t.data_ptr() + (1 << 40) * r for r in range(1)]
+
+    monkeypatch.setattr(symm, "empty", lambda n, dtype, device: torch.empty(n, dtype=dtype))
+    monkeypatch.setattr(symm, "rendezvous", lambda t, group: FakeHandle(t))
+    tdist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                             world_size=1)
+    try:
+        for out_dtype, names in (("bf16", ["x", "idx", "w", "partial"]),
+                                 ("fp8", ["x", "scale", "idx", "w", "partial"])):
+            g = ep.EpGroup(E=32, k=4, H=256, max_tokens=10, out_dtype=out_dtype, device="cpu")
+            assert g.G == 1 and g.capacity == 10
+            base = g._raw.data_ptr()
+            spans = []
+            for name in names:
+                t = getattr(g.bufs, name)
+                off = t.data_ptr() - base
+                assert off % 256 == 0 and g.peer_addr[0][name] == base + off
+                spans.append((off, off + t.numel() * t.element_size()))
+            spans.sort()
+            assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+            assert spans[-1][1] <= g._raw.numel()
+            assert set(g.peer_addr[0]) == set(names)
+    finally:
+        tdist.destroy_process_group()
