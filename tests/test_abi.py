@@ -222,3 +222,37 @@ def test_ep_entries_reject_bad_arguments(tk):
     neg = (ctypes.c_int64 * G)(*[-1] * G)
     assert L.tk_ep_combine(parts, base, neg, FAKE, FAKE, T, G, 256, FAKE, None, None) == 1
     assert L.tk_ep_combine(parts, base, rows, FAKE, FAKE, 0, G, 256, FAKE, None, None) == 0
+
+
+def test_binding_without_library_raises(tmp_path):
+    """A copy of the package without libtk_route.so: importing the binding fails loudly; there is
+    no CPU path to fall back on."""
+    import shutil
+    import subprocess
+    import sys
+
+    pkg = os.path.join(ROOT, "token_routing_gate_b200")
+    dst = tmp_path / "token_routing_gate_b200"
+    dst.mkdir()
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            shutil.copy(os.path.join(pkg, name), dst / name)
+    code = "import token_routing_gate_b200.tk"
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode != 0
+    assert "is not built" in r.stderr and "no CPU path" in r.stderr, r.stderr[-2000:]
+
+
+def test_product_modules_do_not_reach_the_oracle():
+    """The package never imports, loads or runs anything under oracle/."""
+    pkg = os.path.join(ROOT, "token_routing_gate_b200")
+    for name in sorted(os.listdir(pkg)):
+        if name.endswith(".py"):
+            text = open(os.path.join(pkg, name)).read()
+            assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), name
+            assert "tk_oracle" not in text and "liboracle" not in text, name
+    csrc = os.path.join(pkg, "csrc")
+    for name in sorted(os.listdir(csrc)):
+        text = open(os.path.join(csrc, name)).read()
+        assert "oracle" not in text.lower(), name
