@@ -509,12 +509,12 @@ def run_op(args, wl):
         ws = tk._workspace(int(tk.lib.tk_reduce_backward_workspace_bytes(T, k)), dev)
         d_x = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         pad = (R - T * k) * H * 2 + (R * 4 if wl.align > 1 else 0)
-        calls = {
+        calls = {   # name: (call, algorithmic bytes, kernels it launches)
             "reduce_backward": (lambda: tk.reduce_backward(g, y, rm.slot_of, w, E, rm=rm, d_y=d_y, d_w=d_w,
                                                            workspace=ws, stream=stream),
-                                T * H * 2 + 2 * T * k * H * 2 + T * k * (8 + 4 + 64) + pad),
+                                T * H * 2 + 2 * T * k * H * 2 + T * k * (8 + 4 + 64) + pad, 2),
             "expand_backward": (lambda: tk.expand_backward(d_y, rm.slot_of, out=d_x, stream=stream),
-                                T * k * H * 2 + T * k * 4 + T * H * 2),
+                                T * k * H * 2 + T * k * 4 + T * H * 2, 1),
         }
         metric = "reduce + expand backward HBM GB/s vs peak"
     else:
@@ -524,31 +524,60 @@ def run_op(args, wl):
         calls = {
             "balance_stats": (lambda: tk.balance_stats(logits, rm.counts, k, wl.score, workspace=ws, out=P,
                                                        stream=stream),
-                              T * E * 4 + E * 4 + ((T + 63) // 64) * E * 8 * 2 + 3 * E * 4),
-            "tp_mask": (lambda: tk.tp_mask(idx, E, 8, 3, out=masked, stream=stream), T * k * 8),
+                              T * E * 4 + E * 4 + ((T + 63) // 64) * E * 8 * 2 + 3 * E * 4, 2),
+            "tp_mask": (lambda: tk.tp_mask(idx, E, 8, 3, out=masked, stream=stream), T * k * 8, 1),
         }
         metric = "load-balance statistics and TP mask us per call"
     peak, peak_kind = load_peak()
-    out = {}
-    for name, (fn, nbytes) in calls.items():
-        for _ in range(args.warmup):
-            fn()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        torch.cuda.synchronize(dev)
-        ev[0].record(stream)
-        for _ in range(args.steps):
-            fn()
-        ev[1].record(stream)
-        torch.cuda.synchronize(dev)
-        us = ev[0].elapsed_time(ev[1]) * 1e3 / args.steps
-        out[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak}
+    # A call whose bytes fit twice in the 126 MB L2 would find its inputs there when launched back
+    # to back, so such calls are timed one launch at a time after writing a 256 MB buffer; larger
+    # ones run back to back (their own traffic evicts the previous launch's).
+    flush_below = 256 << 20
+    flush = torch.empty(flush_below, dtype=torch.uint8, device=dev)
+    out, l2, launches = {}, {}, 0
+    clocks = ClockSampler(0)
+    with clocks:
+        for name, (fn, nbytes, nk) in calls.items():
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize(dev)
+            if nbytes < flush_below:
+                pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                         for _ in range(args.steps)]
+                for a, b in pairs:
+                    flush.fill_(1)
+                    a.record(stream)
+                    fn()
+                    b.record(stream)
+                torch.cuda.synchronize(dev)
+                us = 1e3 * sum(a.elapsed_time(b) for a, b in pairs) / args.steps
+                l2[name] = "flushed (256 MB written) before each timed launch"
+            else:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                ev[0].record(stream)
+                for _ in range(args.steps):
+                    fn()
+                ev[1].record(stream)
+                torch.cuda.synchronize(dev)
+                us = ev[0].elapsed_time(ev[1]) * 1e3 / args.steps
+                l2[name] = "no flush: %.2f GB per launch (> 126 MB L2)" % (nbytes / 1e9)
+            launches += nk * args.steps
+            out[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak}
     first = next(iter(out))
     line = {"metric": metric, "op": args.op, "value": out[first]["gbs"] if args.op == "backward" else out[first]["us"],
             "unit": "GB/s" if args.op == "backward" else "us", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": args.op == "backward", "dtype": "bf16",
             "data": "synthetic", "config": {"workload": wl.name, "T": T, "E": E, "k": k, "H": H,
-                                             "align": wl.align, "rows_used": R},
-            "peak": peak, "peak_kind": peak_kind, "kernels": out, "gpu_launches": None}
+                                             "align": wl.align, "rows_used": R, "l2": l2},
+            "peak": peak, "peak_kind": peak_kind, "kernels": out, "clocks": clocks.summary(),
+            "gpu_launches": launches}
+    if args.op == "backward":
+        line["roofline"] = {"bound": "hbm", "kernel": "reduce_backward_kernel",
+                            "achieved": out[first]["gbs"], "peak": peak, "peak_kind": peak_kind,
+                            "unit": "GB/s", "frac": out[first]["frac"],
+                            "traffic": ncu_traffic("backward.cu", "reduce_backward_kernel",
+                                                   "backward_" + wl.name),
+                            "algorithmic_bytes_per_launch": out[first]["bytes"]}
     print(json.dumps(line), flush=True)
     return 0
 
