@@ -4,12 +4,15 @@
 // computation). The pages give no formulas; the readings are stated at the C declarations.
 //
 // Balance statistics, deterministic and in double:
-//   balance_partial_kernel: one CTA per tile of 64 tokens, one warp per 8 tokens. Each lane
-//     holds experts lane, lane+32, ... of a token, normalises their unbiased scores over the
-//     row (warp reductions) and adds them into per-lane double accumulators; the CTA then sums
-//     its 8 warps in order and writes one row of a [tiles x E] partial-sum matrix.
-//   balance_final_kernel: one CTA sums each column in tile order, forms P, f and the loss with
-//     a fixed-order tree. The tiling depends on T only, so results do not depend on the GPU.
+//   balance_partial_kernel: one CTA per tile of 64 tokens, one warp per 4 tokens (per 8 when
+//     E > 256, to bound registers). Each lane holds experts lane, lane+32, ... of a token,
+//     normalises their unbiased scores over the row (warp reductions) and adds them into
+//     per-lane double accumulators, loading the next token's logits meanwhile; the CTA then
+//     sums its warps in order and writes one row of a [tiles x E] partial-sum matrix.
+//   balance_final_kernel: one CTA sums each column (up to 8 threads per column, each over a
+//     contiguous range of tiles with 16 loads in flight, the range sums then added in order),
+//     forms P, f and the loss with a fixed-order tree. The grouping depends on T and E only, so
+//     results do not depend on the GPU.
 // Over several data-parallel ranks the same statistics of the whole batch come from
 // tk_balance_score_sums (each rank's column sums, in tile order) + an all-reduce of the sums,
 // the counts and T + tk_balance_finalize (the final kernel over one "tile" of summed values).
@@ -23,9 +26,14 @@ namespace tk {
 namespace {
 
 constexpr int kStatTileTokens = 64;
-constexpr int kStatWarps = 8;
-constexpr int kStatTokensPerWarp = kStatTileTokens / kStatWarps;
 constexpr int kFinalThreads = 1024;
+constexpr int kMaxColumnSplit = 8;
+
+// Warps of a partial CTA: 16 (4 tokens each) while a lane's experts fit in few registers, else 8
+// (8 tokens each). More warps hide the latency of the double exponential's dependent chain; the
+// tile of 64 tokens, and so the partial matrix, is the same either way.
+template <int EPL>
+__host__ __device__ constexpr int stat_warps() { return EPL <= 8 ? 16 : 8; }
 
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
@@ -39,10 +47,72 @@ __device__ __forceinline__ float warp_max_f(float v) {
     return v;
 }
 
+// One token's logits, lane-strided (experts lane, lane+32, ...); -inf past E or past T.
 template <int EPL>
-__global__ void __launch_bounds__(kStatWarps * 32)
+__device__ __forceinline__ void load_logits(const float* __restrict__ logits, int64_t t, int T, int E,
+                                            int lane, float (&l)[EPL]) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        l[i] = (t < T && e < E) ? logits[t * E + e] : -INFINITY;
+    }
+}
+
+// Rows [c0, c1) of column e of a [tiles x E] matrix of doubles, summed in row order. The loads of
+// 16 rows go out together before their additions, so the range costs (c1-c0)/16 memory round
+// trips instead of one per few rows; the additions are those of a plain loop over c.
+__device__ __forceinline__ double column_range_sum(const double* __restrict__ partial, int c0, int c1,
+                                                   int E, int e) {
+    constexpr int kBatch = 16;
+    double sum = 0.0;
+    int c = c0;
+    for (; c + kBatch <= c1; c += kBatch) {
+        double v[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) v[j] = partial[static_cast<int64_t>(c + j) * E + e];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) sum += v[j];
+    }
+    for (; c < c1; ++c) sum += partial[static_cast<int64_t>(c) * E + e];
+    return sum;
+}
+
+// Column sums of a [tiles x E] partial matrix by one CTA of kFinalThreads threads, into
+// out[e] for e < E (shared memory or global). With E small enough, S = min(kFinalThreads / E,
+// kMaxColumnSplit) threads share a column: thread (s, e) sums rows [s*chunk, (s+1)*chunk), and
+// the S range sums are added in order s = 0, 1, ... Every kernel that sums a partial matrix
+// calls this with the same block size, so equal inputs give equal bits; the grouping depends on
+// tiles and E only. Ends with __syncthreads().
+__device__ __forceinline__ void column_sums(const double* __restrict__ partial, int tiles, int E,
+                                            double* __restrict__ split /* [kMaxColumnSplit*E] smem, E <= kFinalThreads */,
+                                            double* __restrict__ out) {
+    int S = kFinalThreads / E;
+    if (S > kMaxColumnSplit) S = kMaxColumnSplit;
+    if (S < 1) S = 1;
+    const int chunk = (tiles + S - 1) / S;
+    for (int i = threadIdx.x; i < S * E; i += blockDim.x) {
+        const int e = i % E;
+        const int sp = i / E;
+        int c0 = sp * chunk, c1 = c0 + chunk;
+        if (c0 > tiles) c0 = tiles;
+        if (c1 > tiles) c1 = tiles;
+        split[sp * E + e] = column_range_sum(partial, c0, c1, E, e);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        double v = 0.0;
+        for (int sp = 0; sp < S; ++sp) v += split[sp * E + e];
+        out[e] = v;
+    }
+    __syncthreads();
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(stat_warps<EPL>() * 32, EPL == 16 ? 2 : 1)
 balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score_fn,
                        double* __restrict__ partial) {
+    constexpr int kStatWarps = stat_warps<EPL>();
+    constexpr int kStatTokensPerWarp = kStatTileTokens / kStatWarps;
     extern __shared__ double wsum[];  // [kStatWarps][E]
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -51,16 +121,15 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
 #pragma unroll
     for (int i = 0; i < EPL; ++i) acc[i] = 0.0;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kStatTileTokens + warp * kStatTokensPerWarp;
+    // the next token's logits are loaded while this token's scores are computed
+    float l[EPL], nxt[EPL];
+    load_logits<EPL>(logits, t0, T, E, lane, l);
     for (int q = 0; q < kStatTokensPerWarp; ++q) {
         const int64_t t = t0 + q;
         if (t >= T) break;
-        const float* row = logits + t * E;
-        float l[EPL];
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int e = i * 32 + lane;
-            l[i] = e < E ? row[e] : -INFINITY;
-        }
+        // (past this warp's last token nothing is loaded: T stands for "no token")
+        load_logits<EPL>(logits, q + 1 < kStatTokensPerWarp ? t + 1 : static_cast<int64_t>(T), T, E,
+                         lane, nxt);
         double s[EPL];
         double z = 0.0;
         if (score_fn == TK_SCORE_SOFTMAX) {
@@ -85,6 +154,8 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
         const double rz = 1.0 / warp_sum_d(z);
 #pragma unroll
         for (int i = 0; i < EPL; ++i) acc[i] += s[i] * rz;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) l[i] = nxt[i];
     }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
@@ -100,18 +171,21 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
     }
 }
 
+static_assert(TK_MAX_EXPERTS <= kFinalThreads, "column_sums' split buffer holds kFinalThreads doubles");
+
 __global__ void __launch_bounds__(kFinalThreads)
 balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_t* __restrict__ counts,
                      int64_t T, int E, int k, float* __restrict__ P, float* __restrict__ f,
                      float* __restrict__ loss) {
+    __shared__ double split[kFinalThreads];
+    __shared__ double sums[TK_MAX_EXPERTS];
     __shared__ double prod[kFinalThreads];
     pdl_wait();
+    column_sums(partial, tiles, E, split, sums);
     // each thread owns experts e = threadIdx.x + i * blockDim.x and keeps their f*P sum
     double mine = 0.0;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        double sum = 0.0;
-        for (int c = 0; c < tiles; ++c) sum += partial[static_cast<int64_t>(c) * E + e];
-        const double Pe = T > 0 ? sum / static_cast<double>(T) : 0.0;
+        const double Pe = T > 0 ? sums[e] / static_cast<double>(T) : 0.0;
         const double fe = T > 0 ? static_cast<double>(E) * counts[e] / (static_cast<double>(k) * static_cast<double>(T)) : 0.0;
         P[e] = static_cast<float>(Pe);
         f[e] = static_cast<float>(fe);
@@ -126,20 +200,18 @@ balance_final_kernel(const double* __restrict__ partial, int tiles, const int32_
     if (threadIdx.x == 0) *loss = static_cast<float>(prod[0]);
 }
 
-// Column sums of the partial matrix in tile order (the same additions as the final kernel).
+// Column sums of the partial matrix (the same additions as the final kernel).
 __global__ void __launch_bounds__(kFinalThreads)
 balance_colsum_kernel(const double* __restrict__ partial, int tiles, int E, double* __restrict__ sums) {
+    __shared__ double split[kFinalThreads];
     pdl_wait();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        double sum = 0.0;
-        for (int c = 0; c < tiles; ++c) sum += partial[static_cast<int64_t>(c) * E + e];
-        sums[e] = sum;
-    }
+    column_sums(partial, tiles, E, split, sums);
 }
 
 template <int EPL>
 cudaError_t launch_partial(const float* logits, int T, int E, int score_fn, double* partial,
                            int tiles, cudaStream_t s) {
+    constexpr int kStatWarps = stat_warps<EPL>();
     const size_t smem = static_cast<size_t>(kStatWarps) * E * sizeof(double);
     static std::atomic<bool> configured[kMaxDevices];
     const int dev = current_device();
