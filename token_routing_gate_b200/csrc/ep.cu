@@ -32,6 +32,11 @@ namespace {
 constexpr uint32_t kEpChunkBytes = 32768;   // bf16 bytes staged per bulk load
 constexpr int kEpFp8Threads = 256;
 constexpr int kEpFp8ChunkChannels = 8192;   // channels quantised per stage
+// Both dispatch kernels stay within the 48 KB of shared memory a CTA gets without an opt-in
+// attribute: the dynamic stage below plus under 1 KB of static barriers and row counts.
+constexpr size_t kEpFp8SmemMax = static_cast<size_t>(kEpFp8ChunkChannels) * 3 + (kEpFp8ChunkChannels / 128) * 4;
+static_assert(kEpChunkBytes + 1024 <= 48 * 1024, "bf16 dispatch stage exceeds the default shared memory");
+static_assert(kEpFp8SmemMax + 1024 <= 48 * 1024, "E4M3 dispatch stage exceeds the default shared memory");
 constexpr int kMaskThreads = 256;
 
 struct EpPeers {
@@ -323,9 +328,6 @@ extern "C" tk_status tk_ep_dispatch(const void* x, const int32_t* topk_idx, cons
     if (out_dtype == TK_OUT_BF16) {
         const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
         const uint32_t smem = min(row_bytes, kEpChunkBytes);
-        err = cudaFuncSetAttribute(ep_dispatch_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(kEpChunkBytes));
-        if (err != cudaSuccess) return check_launch(err, "ep_dispatch_bf16_kernel setup");
         err = launch_pdl(ep_dispatch_bf16_kernel, dim3(T), dim3(32), smem, s,
                          static_cast<const uint8_t*>(x), topk_idx, topk_w, dest_slot, send_offsets, E,
                          k, G, row_bytes, p, err_flag);
@@ -333,10 +335,6 @@ extern "C" tk_status tk_ep_dispatch(const void* x, const int32_t* topk_idx, cons
     }
     const int chunk = H < kEpFp8ChunkChannels ? H : kEpFp8ChunkChannels;
     const size_t smem = static_cast<size_t>(chunk) * 3 + static_cast<size_t>(chunk / 128) * 4;
-    const size_t smem_max = static_cast<size_t>(kEpFp8ChunkChannels) * 3 + (kEpFp8ChunkChannels / 128) * 4;
-    err = cudaFuncSetAttribute(ep_dispatch_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem_max));
-    if (err != cudaSuccess) return check_launch(err, "ep_dispatch_fp8_kernel setup");
     err = launch_pdl(ep_dispatch_fp8_kernel, dim3(T), dim3(kEpFp8Threads), smem, s,
                      static_cast<const uint16_t*>(x), topk_idx, topk_w, dest_slot, send_offsets, E, k,
                      G, H, p, err_flag);
