@@ -14,8 +14,14 @@ pytestmark = pytest.mark.gpu
 ULP32 = 2.0 ** -23  # both sides accumulate in double; the fp32 outputs differ by rounding only
 
 
+# E=300 and E=1024 take the partial kernel's 8-warp forms (shared memory above 48 KB at 1024)
+# and the final sums' uneven (3 threads per column) and unsplit (1 per column) forms
+LARGE_E = [W.V3.with_(T=515, E=300, k=6, name="T515_E300_k6_sigmoid_bias"),
+           W.MID.with_(T=333, E=1024, k=8, name="T333_E1024_k8_softmax")]
+
+
 @pytest.mark.parametrize("wl", [W.V3, W.MID, W.TINY.with_(T=77, E=37, k=5),
-                                W.SKEW.with_(T=1000)], ids=lambda w: w.name)
+                                W.SKEW.with_(T=1000), *LARGE_E], ids=lambda w: w.name)
 def test_balance_stats(wl):
     logits, bias = W.gate_inputs(wl, "cuda")
     idx, _ = tk.gate_topk(logits, wl.k, wl.score, bias)
@@ -38,7 +44,7 @@ def test_balance_stats_empty_batch():
     assert (P == 0).all() and (f == 0).all() and loss.item() == 0.0
 
 
-@pytest.mark.parametrize("wl", [W.MID, W.V3.with_(T=3000)], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [W.MID, W.V3.with_(T=3000), *LARGE_E], ids=lambda w: w.name)
 def test_balance_sums_then_finalize_is_the_one_call(wl):
     logits, bias = W.gate_inputs(wl, "cuda")
     idx, _ = tk.gate_topk(logits, wl.k, wl.score, bias)
