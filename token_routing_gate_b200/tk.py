@@ -5,6 +5,11 @@ every step runs in the library's kernels. The names follow the C entry points wi
 ``tk_`` prefix. Missing outputs are allocated with torch (caching allocator) before the call;
 pass preallocated tensors to keep allocation out of a timed loop. There is no fallback: if the
 library is not built, importing this module raises.
+
+Every tensor handed to the library is checked first: on a CUDA device, contiguous, of the dtype
+the C declaration names, and holding at least the elements the call reads or writes (a smaller
+output would otherwise be written past its end). A failed check raises ValueError or TypeError
+before anything runs; the library's own argument checks then raise TkError.
 """
 import ctypes
 import os
@@ -114,12 +119,42 @@ def _check(fn, status):
         raise TkError(fn, lib.tk_status_str(status).decode(), lib.tk_last_error_detail().decode())
 
 
-def _ptr(t):
+F32, F64, I32, BF16, U8 = torch.float32, torch.float64, torch.int32, torch.bfloat16, torch.uint8
+E4M3 = (torch.uint8, torch.float8_e4m3fn)     # E4M3 codes: raw bytes or torch's fp8 type
+
+
+def _ptr(t, dtype=None, numel=0, name="tensor"):
+    """Device address of a tensor for the library (None stays NULL). The tensor must be on a CUDA
+    device and contiguous; `dtype` (one dtype or a tuple) and `numel` (the fewest elements the
+    call touches) are checked when given."""
     if t is None:
         return None
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device, not {t.device}")
+    if dtype is not None:
+        ok = dtype if isinstance(dtype, tuple) else (dtype,)
+        if t.dtype not in ok:
+            raise TypeError(f"{name} must be {' or '.join(str(d) for d in ok)}, not {t.dtype}")
     if not t.is_contiguous():
-        raise ValueError("tensors passed to libtk_route must be contiguous")
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call needs {numel}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _shape2(t, name):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return t.shape
+
+
+def _flag(err_flag):
+    return _ptr(err_flag, I32, 1, "err_flag")
+
+
+def _ws(workspace, nbytes):
+    """Workspaces are byte tensors: their numel() is passed as the byte count."""
+    return _ptr(workspace, U8, nbytes, "workspace")
 
 
 def _stream(stream):
@@ -139,14 +174,15 @@ def route_map_workspace_bytes(T, E, k):
 def gate_topk(logits, k, score="sigmoid", bias=None, renormalize=True, topk_idx=None, topk_w=None,
               stream=None):
     """logits fp32 [T,E] -> (topk_idx int32 [T,k], topk_w fp32 [T,k])."""
-    T, E = logits.shape
+    T, E = _shape2(logits, "logits")
     if topk_idx is None:
         topk_idx = torch.empty(T, k, dtype=torch.int32, device=logits.device)
     if topk_w is None:
         topk_w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
-    _check("tk_gate_topk", lib.tk_gate_topk(_ptr(logits), _ptr(bias), T, E, k, SCORE[score],
-                                            int(bool(renormalize)), _ptr(topk_idx), _ptr(topk_w),
-                                            _stream(stream)))
+    _check("tk_gate_topk", lib.tk_gate_topk(_ptr(logits, F32, T * E, "logits"), _ptr(bias, F32, E, "bias"),
+                                            T, E, k, SCORE[score], int(bool(renormalize)),
+                                            _ptr(topk_idx, I32, T * k, "topk_idx"),
+                                            _ptr(topk_w, F32, T * k, "topk_w"), _stream(stream)))
     return topk_idx, topk_w
 
 
@@ -160,7 +196,7 @@ class RouteMap:
 
 
 def route_map(topk_idx, E, align=1, out=None, err_flag=None, stream=None):
-    T, k = topk_idx.shape
+    T, k = _shape2(topk_idx, "topk_idx")
     dev = topk_idx.device
     if out is None:
         ws = max(route_map_workspace_bytes(T, E, k), 16)
@@ -170,36 +206,42 @@ def route_map(topk_idx, E, align=1, out=None, err_flag=None, stream=None):
                        torch.empty(max(max_rows(T, E, k, align), 1), dtype=torch.int32, device=dev),
                        torch.empty((ws + 15) // 16, 16, dtype=torch.uint8, device=dev), align)
     _check("tk_route_map", lib.tk_route_map(
-        _ptr(topk_idx), T, E, k, align, _ptr(out.counts), _ptr(out.offsets), _ptr(out.slot_of),
-        _ptr(out.token_of), _ptr(out.workspace), out.workspace.numel(), _ptr(err_flag),
+        _ptr(topk_idx, I32, T * k, "topk_idx"), T, E, k, align, _ptr(out.counts, I32, E, "counts"),
+        _ptr(out.offsets, I32, E + 1, "offsets"), _ptr(out.slot_of, I32, T * k, "slot_of"),
+        _ptr(out.token_of, I32, max_rows(T, E, k, align), "token_of"),
+        _ws(out.workspace, route_map_workspace_bytes(T, E, k)), out.workspace.numel(), _flag(err_flag),
         _stream(stream)))
     return out
 
 
 def expand(x, rm, E, k, out_dtype="bf16", out=None, out_scale=None, err_flag=None, stream=None):
     """x bf16 [T,H] -> out [max_rows, H] (bf16, or E4M3 as uint8 with fp32 scales [max_rows, H/128])."""
-    T, H = x.shape
-    R = max(max_rows(T, E, k, rm.align), 1)
+    T, H = _shape2(x, "x")
+    R_max = max_rows(T, E, k, rm.align)
+    R = max(R_max, 1)
     if out is None:
         out = torch.empty(R, H, dtype=torch.bfloat16 if out_dtype == "bf16" else torch.uint8,
                           device=x.device)
     if out_dtype == "fp8" and out_scale is None:
         out_scale = torch.empty(R, H // 128, dtype=torch.float32, device=x.device)
     _check("tk_expand", lib.tk_expand(
-        _ptr(x), _ptr(rm.slot_of), _ptr(rm.offsets), _ptr(rm.token_of), T, E, k, H, rm.align,
-        OUT_DTYPE[out_dtype], _ptr(out), _ptr(out_scale), _ptr(err_flag), _stream(stream)))
+        _ptr(x, BF16, T * H, "x"), _ptr(rm.slot_of, I32, T * k, "slot_of"),
+        _ptr(rm.offsets, I32, E + 1, "offsets"), _ptr(rm.token_of, I32, R_max, "token_of"), T, E, k, H,
+        rm.align, OUT_DTYPE[out_dtype], _ptr(out, E4M3 if out_dtype == "fp8" else BF16, R_max * H, "out"),
+        _ptr(out_scale, F32, R_max * (H // 128), "out_scale"), _flag(err_flag), _stream(stream)))
     return (out, out_scale) if out_dtype == "fp8" else out
 
 
 def reduce(y, slot_of, w=None, out=None, err_flag=None, stream=None, masked=False):
     """y bf16 [rows,H], slot_of int32 [T,k], w fp32 [T,k] or None -> out bf16 [T,H].
     masked=True calls tk_reduce_masked (same results; faster when most pairs are -1)."""
-    T, k = slot_of.shape
-    H = y.shape[1]
+    T, k = _shape2(slot_of, "slot_of")
+    rows, H = _shape2(y, "y")
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device)
     fn, name = (lib.tk_reduce_masked, "tk_reduce_masked") if masked else (lib.tk_reduce, "tk_reduce")
-    _check(name, fn(_ptr(y), y.shape[0], _ptr(slot_of), _ptr(w), T, k, H, _ptr(out), _ptr(err_flag),
+    _check(name, fn(_ptr(y, BF16, rows * H, "y"), rows, _ptr(slot_of, I32, T * k, "slot_of"),
+                    _ptr(w, F32, T * k, "w"), T, k, H, _ptr(out, BF16, T * H, "out"), _flag(err_flag),
                     _stream(stream)))
     return out
 
@@ -210,32 +252,35 @@ def _workspace(nbytes, device):
 
 def balance_stats(logits, counts, k, score="sigmoid", workspace=None, out=None, stream=None):
     """Load-balance statistics -> (P fp32 [E], f fp32 [E], loss fp32 [1])."""
-    T, E = logits.shape
+    T, E = _shape2(logits, "logits")
     dev = counts.device
+    ws_bytes = int(lib.tk_balance_stats_workspace_bytes(T, E))
     if workspace is None:
-        workspace = _workspace(int(lib.tk_balance_stats_workspace_bytes(T, E)), dev)
+        workspace = _workspace(ws_bytes, dev)
     if out is None:
         out = (torch.empty(E, dtype=torch.float32, device=dev),
                torch.empty(E, dtype=torch.float32, device=dev),
                torch.empty(1, dtype=torch.float32, device=dev))
     P, f, loss = out
     _check("tk_balance_stats", lib.tk_balance_stats(
-        _ptr(logits), _ptr(counts), T, E, k, SCORE[score], _ptr(P), _ptr(f), _ptr(loss),
-        _ptr(workspace), workspace.numel(), _stream(stream)))
+        _ptr(logits, F32, T * E, "logits"), _ptr(counts, I32, E, "counts"), T, E, k, SCORE[score],
+        _ptr(P, F32, E, "P"), _ptr(f, F32, E, "f"), _ptr(loss, F32, 1, "loss"),
+        _ws(workspace, ws_bytes), workspace.numel(), _stream(stream)))
     return P, f, loss
 
 
 def balance_score_sums(logits, score="sigmoid", workspace=None, out=None, stream=None):
     """Per-expert sums (double [E]) of the normalised unbiased scores over this batch's tokens."""
-    T, E = logits.shape
+    T, E = _shape2(logits, "logits")
     dev = logits.device
+    ws_bytes = int(lib.tk_balance_stats_workspace_bytes(T, E))
     if workspace is None:
-        workspace = _workspace(int(lib.tk_balance_stats_workspace_bytes(T, E)), dev)
+        workspace = _workspace(ws_bytes, dev)
     if out is None:
         out = torch.empty(E, dtype=torch.float64, device=dev)
     _check("tk_balance_score_sums", lib.tk_balance_score_sums(
-        _ptr(logits), T, E, SCORE[score], _ptr(out), _ptr(workspace), workspace.numel(),
-        _stream(stream)))
+        _ptr(logits, F32, T * E, "logits"), T, E, SCORE[score], _ptr(out, F64, E, "sums"),
+        _ws(workspace, ws_bytes), workspace.numel(), _stream(stream)))
     return out
 
 
@@ -247,17 +292,18 @@ def balance_finalize(sums, counts, T_total, k, out=None, stream=None):
         out = (torch.empty(E, device=dev), torch.empty(E, device=dev), torch.empty(1, device=dev))
     P, f, loss = out
     _check("tk_balance_finalize", lib.tk_balance_finalize(
-        _ptr(sums), _ptr(counts), int(T_total), E, k, _ptr(P), _ptr(f), _ptr(loss), _stream(stream)))
+        _ptr(sums, F64, E, "sums"), _ptr(counts, I32, E, "counts"), int(T_total), E, k,
+        _ptr(P, F32, E, "P"), _ptr(f, F32, E, "f"), _ptr(loss, F32, 1, "loss"), _stream(stream)))
     return P, f, loss
 
 
 def tp_mask(topk_idx, E, tp_size, tp_rank, out=None, stream=None):
     """Keep this rank's experts (renumbered locally), mark the rest -1."""
-    T, k = topk_idx.shape
+    T, k = _shape2(topk_idx, "topk_idx")
     if out is None:
         out = torch.empty_like(topk_idx)
-    _check("tk_tp_mask", lib.tk_tp_mask(_ptr(topk_idx), T, k, E, tp_size, tp_rank, _ptr(out),
-                                        _stream(stream)))
+    _check("tk_tp_mask", lib.tk_tp_mask(_ptr(topk_idx, I32, T * k, "topk_idx"), T, k, E, tp_size, tp_rank,
+                                        _ptr(out, I32, T * k, "out"), _stream(stream)))
     return out
 
 
@@ -265,51 +311,57 @@ def reduce_backward(grad_out, y, slot_of, w, E, rm=None, d_y=None, d_w=None, wor
                     err_flag=None, stream=None):
     """Backward of reduce -> (d_y bf16 [rows, H], d_w fp32 [T, k]). With a RouteMap `rm`,
     padding rows of d_y are zeroed."""
-    T, k = slot_of.shape
-    H = grad_out.shape[1]
+    T, k = _shape2(slot_of, "slot_of")
+    H = _shape2(grad_out, "grad_out")[1]
+    rows = _shape2(y, "y")[0]
     dev = grad_out.device
     if d_y is None:
         d_y = torch.empty_like(y)
     if d_w is None:
         d_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ws_bytes = int(lib.tk_reduce_backward_workspace_bytes(T, k))
     if workspace is None:
-        workspace = _workspace(int(lib.tk_reduce_backward_workspace_bytes(T, k)), dev)
+        workspace = _workspace(ws_bytes, dev)
     _check("tk_reduce_backward", lib.tk_reduce_backward(
-        _ptr(grad_out), _ptr(y), y.shape[0], _ptr(slot_of),
-        _ptr(rm.offsets) if rm is not None else None, _ptr(rm.token_of) if rm is not None else None,
-        _ptr(w), T, E, k, H, _ptr(d_y), _ptr(d_w), _ptr(workspace), workspace.numel(),
-        _ptr(err_flag), _stream(stream)))
+        _ptr(grad_out, BF16, T * H, "grad_out"), _ptr(y, BF16, rows * H, "y"), rows,
+        _ptr(slot_of, I32, T * k, "slot_of"),
+        _ptr(rm.offsets, I32, E + 1, "offsets") if rm is not None else None,
+        _ptr(rm.token_of, I32, max_rows(T, E, k, rm.align), "token_of") if rm is not None else None,
+        _ptr(w, F32, T * k, "w"), T, E, k, H, _ptr(d_y, BF16, rows * H, "d_y"),
+        _ptr(d_w, F32, T * k, "d_w"), _ws(workspace, ws_bytes), workspace.numel(),
+        _flag(err_flag), _stream(stream)))
     return d_y, d_w
 
 
 def expand_backward(d_xe, slot_of, out=None, err_flag=None, stream=None):
     """Backward of a bf16 expand: d_x[t] = sum_j d_xe[slot_of[t, j]]."""
-    T, k = slot_of.shape
-    H = d_xe.shape[1]
+    T, k = _shape2(slot_of, "slot_of")
+    rows, H = _shape2(d_xe, "d_xe")
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=d_xe.device)
     _check("tk_expand_backward", lib.tk_expand_backward(
-        _ptr(d_xe), d_xe.shape[0], _ptr(slot_of), T, k, H, _ptr(out), _ptr(err_flag),
-        _stream(stream)))
+        _ptr(d_xe, BF16, rows * H, "d_xe"), rows, _ptr(slot_of, I32, T * k, "slot_of"), T, k, H,
+        _ptr(out, BF16, T * H, "out"), _flag(err_flag), _stream(stream)))
     return out
 
 
 def selftest_bounded_wait(limit_ns, err_flag, stream=None):
     """Run the bounded-wait self-test kernel (it always times out and flags DEVERR_TIMEOUT)."""
-    _check("tk_selftest_bounded_wait", lib.tk_selftest_bounded_wait(int(limit_ns), _ptr(err_flag),
+    _check("tk_selftest_bounded_wait", lib.tk_selftest_bounded_wait(int(limit_ns), _flag(err_flag),
                                                                     _stream(stream)))
 
 
 # ---------------------------------------------------------------- expert-parallel dispatch / combine
-def _addr(t):
-    """Device address of a tensor (contiguous) or a raw integer address (e.g. a peer's buffer)."""
+def _addr(t, dtype=None, rows=0, name="buffer"):
+    """Device address of a tensor, or a raw integer address (e.g. a peer's buffer, which only its
+    owner can check). A tensor is checked as by _ptr and must have at least `rows` rows."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
-    if not t.is_contiguous():
-        raise ValueError("tensors passed to libtk_route must be contiguous")
-    return t.data_ptr()
+    if t.dim() < 1 or t.shape[0] < rows:
+        raise ValueError(f"{name} has shape {tuple(t.shape)}; the call needs {rows} rows")
+    return _ptr(t, dtype, 0, name).value
 
 
 class EpLayout:
@@ -321,7 +373,7 @@ class EpLayout:
 
 
 def ep_layout(topk_idx, E, G, out=None, err_flag=None, stream=None):
-    T, k = topk_idx.shape
+    T, k = _shape2(topk_idx, "topk_idx")
     dev = topk_idx.device
     if out is None:
         out = EpLayout(torch.empty(G, dtype=torch.int32, device=dev),
@@ -330,29 +382,34 @@ def ep_layout(topk_idx, E, G, out=None, err_flag=None, stream=None):
                        torch.empty(T * G, dtype=torch.int32, device=dev),
                        _workspace(int(lib.tk_ep_layout_workspace_bytes(T, G)), dev), G)
     _check("tk_ep_layout", lib.tk_ep_layout(
-        _ptr(topk_idx), T, E, k, G, _ptr(out.send_counts), _ptr(out.send_offsets),
-        _ptr(out.dest_slot), _ptr(out.send_token), _ptr(out.workspace), out.workspace.numel(),
-        _ptr(err_flag), _stream(stream)))
+        _ptr(topk_idx, I32, T * k, "topk_idx"), T, E, k, G, _ptr(out.send_counts, I32, G, "send_counts"),
+        _ptr(out.send_offsets, I32, G + 1, "send_offsets"), _ptr(out.dest_slot, I32, T * G, "dest_slot"),
+        _ptr(out.send_token, I32, T * G, "send_token"),
+        _ws(out.workspace, int(lib.tk_ep_layout_workspace_bytes(T, G))), out.workspace.numel(),
+        _flag(err_flag), _stream(stream)))
     return out
 
 
 def ep_peer(x, idx, w, base_row, rows, scale=None):
     """Descriptor of one destination's receive buffers: tensors or raw device addresses."""
-    return EpPeer(_addr(x), _addr(scale), _addr(idx), _addr(w), int(base_row), int(rows))
+    rows = int(rows)
+    return EpPeer(_addr(x, (BF16,) + E4M3, rows, "x"), _addr(scale, F32, rows, "scale"),
+                  _addr(idx, I32, rows, "idx"), _addr(w, F32, rows, "w"), int(base_row), rows)
 
 
 def ep_dispatch(x, topk_idx, topk_w, layout, E, peers, out_dtype="bf16", err_flag=None,
                 stream=None):
     """Writes this rank's tokens into the G destinations' receive buffers (peers: G EpPeer)."""
-    T, H = x.shape
-    k = topk_idx.shape[1]
+    T, H = _shape2(x, "x")
+    k = _shape2(topk_idx, "topk_idx")[1]
     G = layout.G
     if len(peers) != G:
         raise ValueError(f"{len(peers)} peer descriptors for G={G}")
     arr = (EpPeer * G)(*peers)
     _check("tk_ep_dispatch", lib.tk_ep_dispatch(
-        _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(layout.dest_slot), _ptr(layout.send_offsets),
-        T, E, k, H, G, OUT_DTYPE[out_dtype], arr, _ptr(err_flag), _stream(stream)))
+        _ptr(x, BF16, T * H, "x"), _ptr(topk_idx, I32, T * k, "topk_idx"), _ptr(topk_w, F32, T * k, "topk_w"),
+        _ptr(layout.dest_slot, I32, T * G, "dest_slot"), _ptr(layout.send_offsets, I32, G + 1, "send_offsets"),
+        T, E, k, H, G, OUT_DTYPE[out_dtype], arr, _flag(err_flag), _stream(stream)))
 
 
 def ep_combine(partials, base_rows, rows, layout, H, out=None, err_flag=None, stream=None):
@@ -362,10 +419,14 @@ def ep_combine(partials, base_rows, rows, layout, H, out=None, err_flag=None, st
     T = layout.dest_slot.shape[0]
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=layout.dest_slot.device)
-    ptrs = (ctypes.c_void_p * G)(*[_addr(p) for p in partials])
+    if len(partials) != G or len(base_rows) != G or len(rows) != G:
+        raise ValueError(f"partials, base_rows and rows need G={G} entries each")
+    ptrs = (ctypes.c_void_p * G)(*[_addr(p, BF16, int(r), f"partials[{d}]")
+                                   for d, (p, r) in enumerate(zip(partials, rows))])
     base = (ctypes.c_int64 * G)(*[int(b) for b in base_rows])
     nrows = (ctypes.c_int64 * G)(*[int(r) for r in rows])
     _check("tk_ep_combine", lib.tk_ep_combine(
-        ptrs, base, nrows, _ptr(layout.dest_slot), _ptr(layout.send_offsets), T, G, H, _ptr(out),
-        _ptr(err_flag), _stream(stream)))
+        ptrs, base, nrows, _ptr(layout.dest_slot, I32, T * G, "dest_slot"),
+        _ptr(layout.send_offsets, I32, G + 1, "send_offsets"), T, G, H, _ptr(out, BF16, T * H, "out"),
+        _flag(err_flag), _stream(stream)))
     return out
