@@ -207,8 +207,10 @@ int tko_gate_topk(const float* logits, const float* bias, int T, int E, int k, i
         }
         double denom = 1.0;
         if (renormalize) {
+#if TKO_PLANT != 17
             denom = 0.0;
             for (int j = 0; j < k; ++j) denom += s[j];
+#endif  /* (plant 17: the renormalisation is skipped) */
         }
         for (int j = 0; j < k; ++j) {
             topk_idx[static_cast<int64_t>(t) * k + j] = order[j];
@@ -254,7 +256,11 @@ int tko_route_map(const int32_t* topk_idx, int T, int E, int k, int align, int32
 #endif
         offsets[e + 1] = offsets[e] + padded;
     }
+#if TKO_PLANT == 18
+    for (int64_t r = 0; r < rmax; ++r) token_of[r] = 0;   /* planted: padding rows name token 0 */
+#else
     for (int64_t r = 0; r < rmax; ++r) token_of[r] = -1;
+#endif
     std::vector<int32_t> fill(E, 0);
     for (int64_t p = 0; p < pairs; ++p) {
         const int e = topk_idx[p];
@@ -282,11 +288,15 @@ int tko_quantize_row_e4m3(const uint16_t* xrow, int H, uint8_t* q, float* scales
     for (int b = 0; b < H / 128; ++b) {
         float amax = 0.0f;
         for (int c = 0; c < 128; ++c) amax = std::max(amax, std::fabs(bf16_to_float(xrow[b * 128 + c])));
+#if TKO_PLANT == 20
+        if (amax == 0.0f) amax = 1e-30f;  /* planted: an epsilon guard instead of scale 0 */
+#else
         if (amax == 0.0f) {
             scales[b] = 0.0f;
             for (int c = 0; c < 128; ++c) q[b * 128 + c] = 0x00;
             continue;
         }
+#endif
 #if TKO_PLANT == 7
         const float scale = amax / 447.0f;  /* planted: wrong E4M3 maximum */
 #else
@@ -432,6 +442,8 @@ int tko_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size, int t
         const int e = topk_idx[p];
 #if TKO_PLANT == 12
         out_idx[p] = (e >= lo && e < lo + el) ? e : -1;  /* planted: not renumbered */
+#elif TKO_PLANT == 19
+        out_idx[p] = (e >= lo && e <= lo + el) ? e - lo : -1;  /* planted: inclusive upper bound */
 #else
         out_idx[p] = (e >= lo && e < lo + el) ? e - lo : -1;
 #endif
@@ -469,7 +481,11 @@ int tko_reduce_backward(const uint16_t* grad_out, const uint16_t* y, int64_t y_r
             for (int c = 0; c < H; ++c) {
                 const float gc = bf16_to_float(g[c]);
                 dot += static_cast<double>(gc) * static_cast<double>(bf16_to_float(y[slot * H + c]));
+#if TKO_PLANT == 21
+                d_y[slot * H + c] = tko_bf16_rne(bf16_to_float(tko_bf16_rne(wj)) * gc);  /* planted: w rounded to bf16 first */
+#else
                 d_y[slot * H + c] = tko_bf16_rne(wj * gc);
+#endif
             }
 #if TKO_PLANT == 11
             d_w[p] = static_cast<float>(dot * wj);  /* planted: weighted dot product */

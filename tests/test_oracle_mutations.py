@@ -3,7 +3,9 @@ tie-break, biased weights, an off-by-one padding, unstable slots, the wrong E4M3
 scale, the wrong reduction order, truncating bf16 rounding, a missing factor in the balance
 loss, a weighted gradient, an un-renumbered TP mask, the expert-parallel combine in the wrong
 rank order, experts dealt round-robin over ranks, global expert ids sent, inclusive receive
-bases) is compiled into a copy of the oracle,
+bases, skipped renormalisation, padding rows naming token 0, an inclusive TP-group bound, an
+epsilon guard in place of the zero scale of an all-zero FP8 block, a gradient weight rounded to
+bf16 first) is compiled into a copy of the oracle,
 and the pins that cover that step must fail against it. The unplanted build must pass them."""
 import os
 import subprocess
@@ -32,6 +34,11 @@ MUTATIONS = {
     14: "ep_layout or ep_dispatch",
     15: "ep_dispatch",
     16: "ep_recv_bases or ep_hand_case",
+    17: "gate_softmax_weights_library or sigmoid_weights_library or gate_all_equal",
+    18: "route_map",
+    19: "tp_mask",
+    20: "fp8",
+    21: "reduce_backward",
 }
 
 
