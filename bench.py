@@ -181,6 +181,27 @@ def cpu_threads():
     return 1  # the oracle is single-threaded C++
 
 
+def system_info(dev=None):
+    """Host core count and CPU model, and the GPU's name when a device is given. Never raises:
+    what cannot be read is None."""
+    info = {"nproc": os.cpu_count(), "cpu_model": None, "gpu_name": None}
+    try:
+        with open("/proc/cpuinfo") as f:
+            for row in f:
+                if row.startswith("model name"):
+                    info["cpu_model"] = row.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    if dev is not None:
+        try:
+            import torch
+            info["gpu_name"] = torch.cuda.get_device_name(dev)
+        except Exception:  # noqa: BLE001  (a name is context, never a reason to fail the run)
+            pass
+    return info
+
+
 def oracle_step(wl, lg, b, x_bits, y_bits):
     """The whole path on the CPU oracle for one sample batch."""
     import oracle
@@ -259,6 +280,7 @@ def run_reference(args, wl):
                                    f"{wl.name}, single-threaded C++ oracle"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
+        "system": system_info(),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -412,6 +434,7 @@ def run_tk(args, wl):
         "kernel_pass_ms_per_step": evented_ms,
         "clocks": clocks.summary(),
         "gpu_launches": launches_per_step * K,
+        "system": system_info(dev),
     }
 
     if not args.no_e2e:
@@ -570,7 +593,7 @@ def run_op(args, wl):
             "data": "synthetic", "config": {"workload": wl.name, "T": T, "E": E, "k": k, "H": H,
                                              "align": wl.align, "rows_used": R, "l2": l2},
             "peak": peak, "peak_kind": peak_kind, "kernels": out, "clocks": clocks.summary(),
-            "gpu_launches": launches}
+            "gpu_launches": launches, "system": system_info(dev)}
     if args.op == "backward":
         line["roofline"] = {"bound": "hbm", "kernel": "reduce_backward_kernel",
                             "achieved": out[first]["gbs"], "peak": peak, "peak_kind": peak_kind,
@@ -685,7 +708,7 @@ def run_ep(args, wl):
             "hbm_gbs": {"dispatch": disp_bytes / (phase_us["dispatch"] * 1e3),
                         "combine": comb_bytes / (phase_us["combine"] * 1e3)},
             "bytes": {"dispatch": disp_bytes, "combine": comb_bytes},
-            "clocks": clocks.summary(), "gpu_launches": None}
+            "clocks": clocks.summary(), "gpu_launches": None, "system": system_info(dev)}
     print(json.dumps(line), flush=True)
     return 0
 

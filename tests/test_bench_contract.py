@@ -38,6 +38,8 @@ def test_reference_arm_line_has_the_contract_keys():
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    sysinfo = line["system"]
+    assert sysinfo["nproc"] >= 1 and "cpu_model" in sysinfo and sysinfo["gpu_name"] is None
 
 
 def test_reference_arm_other_ranks_exit_quietly():
