@@ -81,7 +81,11 @@ def pipeline(monkeypatch):
     monkeypatch.setattr(P.torch.cuda, "Event", FakeEvent)
     monkeypatch.setattr(P.torch.cuda, "current_stream", lambda *a: caller)
     monkeypatch.setattr(P.torch.cuda, "current_device", lambda: 0)
+    kept = []
+    monkeypatch.setattr(P, "_keep_for", lambda stream, *ts: kept.append(
+        (stream.name, [t for t in ts if t is not None])))
     pipe = P.RoutingPipeline(T=8, E=4, k=2, device="cpu")
+    pipe.kept = kept
     return pipe, caller, calls
 
 
@@ -124,3 +128,19 @@ def test_ready_event_is_waited_for_before_the_gate(pipeline):
     log = pipe.stream.log
     assert log.index(("wait", ready.id)) < log.index(("gate", id(h.idx)))
     assert log[-1] == ("record", h.event.id)
+
+
+def test_caller_tensors_are_kept_alive_for_the_streams_that_use_them(pipeline):
+    pipe, caller, calls = pipeline
+    # construction: every tensor of both sets is marked for the routing stream
+    assert [k[0] for k in pipe.kept] == ["routing", "routing"]
+    assert all(len(k[1]) == 7 for k in pipe.kept)
+    pipe.kept.clear()
+    h = pipe.route("logits", bias="bias", err_flag="flag")
+    assert pipe.kept == [("routing", ["logits", "bias", "flag"])]
+    pipe.kept.clear()
+    pipe.dispatch_combine(h, "x", "y", "out", "xe")          # the current stream: nothing to do
+    assert pipe.kept == []
+    other = FakeStream("other")
+    pipe.dispatch_combine(h, "x", "y", "out", "xe", xs="xs", stream=other)
+    assert pipe.kept == [("other", ["x", "y", "out", "xe", "xs"])]

@@ -18,10 +18,22 @@ and records an event; `dispatch_combine` makes the caller's stream wait for that
 runs expand and reduce. A set is reused only after the reduce that read it has finished. The
 routing stream does not wait for the caller's stream: pass `ready` (a CUDA event) when the
 batch's logits are produced on another stream.
+
+Tensors the caller passes in are used on the routing stream (and, for `dispatch_combine`, on
+`stream` when it is not the current one); both calls mark them with `record_stream`, so the
+caching allocator does not hand their memory to anyone else before that work has run, even
+if the caller drops its last reference right after the call.
 """
 import torch
 
 from . import tk
+
+
+def _keep_for(stream, *tensors):
+    """Keep the tensors' memory from being reused until the work queued on `stream` is done."""
+    for t in tensors:
+        if t is not None:
+            t.record_stream(stream)
 
 
 class RouteHandle:
@@ -42,6 +54,9 @@ class RoutingPipeline:
             idx = torch.zeros(T, k, dtype=torch.int32, device=device)
             w = torch.empty(T, k, dtype=torch.float32, device=device)
             rm = tk.route_map(idx, E, align)      # allocates the route-map buffers once
+            # allocated on the current stream, used on ours
+            _keep_for(self.stream, idx, w, rm.counts, rm.offsets, rm.slot_of, rm.token_of,
+                      rm.workspace)
             self.sets.append((idx, w, rm))
         self.done = [None] * depth                # event: the last reduce that read the set
         self.n = 0
@@ -57,6 +72,7 @@ class RoutingPipeline:
             s.wait_event(self.done[slot])
         if ready is not None:
             s.wait_event(ready)
+        _keep_for(s, logits, bias, err_flag)
         tk.gate_topk(logits, self.k, self.score, bias, self.renormalize, idx, w, s)
         tk.route_map(idx, self.E, self.align, out=rm, err_flag=err_flag, stream=s)
         ev = torch.cuda.Event()
@@ -69,6 +85,8 @@ class RoutingPipeline:
         reduce y by its slots and weights into out, on `stream` (default: the current one)."""
         s = stream if stream is not None else torch.cuda.current_stream()
         s.wait_event(h.event)
+        if s != torch.cuda.current_stream():
+            _keep_for(s, x, y, out, xe, xs, err_flag)
         tk.expand(x, h.rm, self.E, self.k, out_dtype, out=xe, out_scale=xs, err_flag=err_flag, stream=s)
         tk.reduce(y, h.rm.slot_of, h.w, out=out, err_flag=err_flag, stream=s)
         ev = torch.cuda.Event()
