@@ -128,7 +128,7 @@ class ClockSampler:
     NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
              0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
-    def __init__(self, index, period_s=0.002):
+    def __init__(self, index, period_s=0.0005):
         self.index, self.period = index, period_s
         self.samples, self.reasons = [], 0
         self.max_mhz = None
@@ -202,15 +202,31 @@ def system_info(dev=None):
     return info
 
 
-def oracle_step(wl, lg, b, x_bits, y_bits):
-    """The whole path on the CPU oracle for one sample batch."""
+def oracle_buffers(wl):
+    """Every output of the oracle's path for one batch of wl, allocated once (outside timing)."""
+    import numpy as np
+    import oracle
+    T, E, k, H = wl.T, wl.E, wl.k, wl.H
+    rmax = oracle.max_rows(T, E, k, wl.align)
+    if wl.out_dtype == "fp8":
+        xe = (np.zeros((rmax, H), np.uint8), np.zeros((rmax, H // 128), np.float32))
+    else:
+        xe = (np.zeros((rmax, H), np.uint16),)
+    return {"gate": (np.empty((T, k), np.int32), np.empty((T, k), np.float32)),
+            "route": (np.empty(E, np.int32), np.empty(E + 1, np.int32), np.empty((T, k), np.int32),
+                      np.empty(rmax, np.int32)),
+            "expand": xe, "reduce": np.empty((T, H), np.uint16)}
+
+
+def oracle_step(wl, lg, b, x_bits, y_bits, bufs):
+    """The whole path on the CPU oracle for one sample batch, into preallocated outputs."""
     import oracle
     fn = oracle.SOFTMAX if wl.score == "softmax" else oracle.SIGMOID
-    idx, w = oracle.gate_topk(lg, b, wl.k, fn)
-    counts, offsets, slot_of, token_of, _ = oracle.route_map(idx, wl.E, wl.align)
+    idx, w = oracle.gate_topk(lg, b, wl.k, fn, out=bufs["gate"])
+    counts, offsets, slot_of, token_of, _ = oracle.route_map(idx, wl.E, wl.align, out=bufs["route"])
     out_dtype = oracle.OUT_FP8_E4M3 if wl.out_dtype == "fp8" else oracle.OUT_BF16
-    oracle.expand(x_bits, slot_of, offsets, wl.E, wl.align, out_dtype)
-    return oracle.reduce(y_bits, slot_of, w)
+    oracle.expand(x_bits, slot_of, offsets, wl.E, wl.align, out_dtype, out=bufs["expand"])
+    return oracle.reduce(y_bits, slot_of, w, out=bufs["reduce"])
 
 
 def oracle_sample_inputs(wl, Ts, seed):
@@ -224,21 +240,26 @@ def oracle_sample_inputs(wl, Ts, seed):
     return sw, lg.numpy(), (b.numpy() if b is not None else None), x, y
 
 
-def time_oracle(wl, seconds, Ts=1024):
+def time_oracle(wl, seconds):
+    """The oracle on the workload's whole batch (T tokens), outputs preallocated, repeated for
+    about `seconds` (at least 3 runs)."""
     from oracle.build import build_oracle
     build_oracle()
+    Ts = wl.T
     sw, lg, b, x, y = oracle_sample_inputs(wl, Ts, wl.seed)
-    oracle_step(sw, lg, b, x, y)  # warm (page in)
+    bufs = oracle_buffers(sw)
+    oracle_step(sw, lg, b, x, y, bufs)  # warm (page in)
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(sw, lg, b, x, y)
+        oracle_step(sw, lg, b, x, y, bufs)
         n += 1
         el = time.perf_counter() - t0
-        if el >= seconds:
+        if el >= seconds and n >= 3:
             break
     return {"value": n * Ts / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{n} runs of the full path on {Ts} tokens of {wl.name} "
-                      f"(E={wl.E}, k={wl.k}, H={wl.H}) in {el:.1f} s, single-threaded C++ oracle"}
+            "sample": f"{n} runs of the full path on the whole {Ts}-token batch of {wl.name} "
+                      f"(E={wl.E}, k={wl.k}, H={wl.H}) in {el:.1f} s, outputs preallocated, "
+                      f"single-threaded C++ oracle"}
 
 
 def run_reference(args, wl):
@@ -250,20 +271,23 @@ def run_reference(args, wl):
     from oracle.build import build_oracle
     build_oracle()
     sw, lg, b, x, y = oracle_sample_inputs(wl, 128, wl.seed)
+    bufs = oracle_buffers(sw)
+    oracle_step(sw, lg, b, x, y, bufs)
     t0 = time.perf_counter()
-    oracle_step(sw, lg, b, x, y)
+    oracle_step(sw, lg, b, x, y, bufs)
     per_token = (time.perf_counter() - t0) / 128
     budget = 120.0 / max(1, args.steps + args.warmup)
     Ts = 64
     while Ts * 2 <= min(wl.T, 8192) and Ts * 2 * per_token <= budget:
         Ts *= 2
     sw, lg, b, x, y = oracle_sample_inputs(wl, Ts, wl.seed)
+    bufs = oracle_buffers(sw)
     for _ in range(args.warmup):
-        oracle_step(sw, lg, b, x, y)
+        oracle_step(sw, lg, b, x, y, bufs)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle_step(sw, lg, b, x, y)
+        oracle_step(sw, lg, b, x, y, bufs)
         times.append(time.perf_counter() - t0)
     total = sum(times)
     value = Ts * args.steps / total
@@ -277,7 +301,7 @@ def run_reference(args, wl):
                    "sample_tokens_per_step": Ts},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": f"{args.steps} steps, each the full path on {Ts} tokens of "
-                                   f"{wl.name}, single-threaded C++ oracle"},
+                                   f"{wl.name} (outputs preallocated), single-threaded C++ oracle"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
         "system": system_info(),
@@ -354,14 +378,17 @@ def run_tk(args, wl):
 
     pipe = RoutingPipeline(wl.T, wl.E, wl.k, wl.score, wl.align, device=dev)
 
-    def pipelined(n):
+    def pipelined(n, step_ends=None):
         """n batches, two in flight: batch i+1's gate + route map on the pipeline's stream while
-        batch i's expand + reduce run on `stream`."""
+        batch i's expand + reduce run on `stream`. step_ends[i], when given, is recorded on
+        `stream` right after batch i's reduce (next to the pipeline's own event there)."""
         pipe.stream.wait_stream(stream)
         h = pipe.route(logits, bias)
         for i in range(n):
             nxt = pipe.route(logits, bias) if i + 1 < n else None
             pipe.dispatch_combine(h, x, y, out, xe, wl.out_dtype, xs, stream=stream)
+            if step_ends is not None:
+                step_ends[i].record(stream)
             h = nxt
 
     for _ in range(args.warmup):
@@ -379,12 +406,24 @@ def run_tk(args, wl):
         dist.barrier(dev_for_collectives)
         return dist.max_over_ranks(start.elapsed_time(end) / 1e3, dev_for_collectives)
 
+    clocks = ClockSampler(dev.index)   # sampled every 0.5 ms over all the passes below
+    clocks.__enter__()
     # Pass 1 (the headline): K batches with two in flight (RoutingPipeline), nothing between the
     # calls, so each kernel's launch also overlaps the end of the previous one.
-    with ClockSampler(dev.index) as clocks:
-        max_s = timed(lambda: pipelined(K))
-    # Pass 1b: the same K steps one after another on one stream (no batch overlap).
+    max_s = timed(lambda: pipelined(K))
+    # Pass 1b: the same K steps one after another on one stream (no batch overlap); this is the
+    # routed tokens/s of all four calls timed as one stream sequence.
     serial_s = timed(lambda: [step() for _ in range(K)])
+    # Pass 1c: the headline's K steps again with an event after every batch's reduce: the
+    # distribution of single step times (median, best, p90) behind the headline's mean.
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    dist.barrier(dev_for_collectives)
+    torch.cuda.synchronize(dev)
+    ends[0].record(stream)
+    pipelined(K, ends[1:])
+    torch.cuda.synchronize(dev)
+    dist.barrier(dev_for_collectives)
+    step_ms = sorted(ends[i].elapsed_time(ends[i + 1]) for i in range(K))
     # Pass 2 (the per-kernel breakdown behind the roofline): the same K steps with events
     # between the calls; the events stop one call's launch from overlapping the previous one.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
@@ -394,6 +433,7 @@ def run_tk(args, wl):
         step(evs[i])
     torch.cuda.synchronize(dev)
     dist.barrier(dev_for_collectives)
+    clocks.__exit__(None, None, None)
     names = ["gate", "route_map", "expand", "reduce"]
     k_ms = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K for j, n in enumerate(names)}
     evented_ms = sum(evs[i][0].elapsed_time(evs[i][4]) for i in range(K)) / K
@@ -408,10 +448,20 @@ def run_tk(args, wl):
                   "reduce": "reduce_kernel"}[dom]
     achieved = kernels[dom]["gbs"]
     er_gbs = (ab["expand"] + ab["reduce"]) / ((k_ms["expand"] + k_ms["reduce"]) / 1e3) / 1e9
+    value = dist.aggregate_rate(wl.T * K, world, max_s)
+    serial_value = dist.aggregate_rate(wl.T * K, world, serial_s)
     line = {
-        "metric": METRIC, "value": dist.aggregate_rate(wl.T * K, world, max_s), "unit": UNIT,
+        "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * max_s / K,
-        "serial": {"value": dist.aggregate_rate(wl.T * K, world, serial_s),
+        "headline_form": "two batches in flight (gate + route map of the next batch overlap "
+                         "expand + reduce of this one); 'serial' is the four calls of every step "
+                         "timed as one stream sequence",
+        "pairs_per_s": wl.k * value,
+        "step_ms": {"mean": 1e3 * max_s / K, "median": statistics.median(step_ms),
+                    "best": step_ms[0], "p90": step_ms[min(K - 1, int(0.9 * K))],
+                    "note": "rank 0's single step times from a repeat of the headline pass with an "
+                            "event after every batch's reduce; mean is the headline's"},
+        "serial": {"value": serial_value, "pairs_per_s": wl.k * serial_value,
                    "ms_per_step": 1e3 * serial_s / K,
                    "note": "the same K steps one after another on one stream"},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",

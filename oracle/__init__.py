@@ -3,7 +3,9 @@
 Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
 import this package. The CUDA library does not use it, and it does not use the CUDA library.
 Arguments are numpy arrays (C-contiguous); bf16 tensors travel as uint16 bit patterns and
-E4M3 codes as uint8. Each wrapper allocates its outputs and returns them.
+E4M3 codes as uint8. Each wrapper allocates its outputs and returns them, unless the caller
+passes them in `out` (arrays of the exact shape and dtype, reused as they are: a timing loop can
+then keep allocation out of what it measures).
 """
 import ctypes
 import os
@@ -110,12 +112,22 @@ def max_rows(T, E, k, align):
     return int(lib().tko_max_rows(T, E, k, align))
 
 
-def gate_topk(logits, bias, k, score_fn, renormalize=True):
+def _outputs(out, *specs):
+    """The caller's output arrays (checked against (shape, dtype) specs), or new ones."""
+    if out is None:
+        return [np.empty(shape, dtype=dt) for shape, dt in specs]
+    out = list(out)
+    for a, (shape, dt) in zip(out, specs):
+        if a.shape != tuple(shape) or a.dtype != np.dtype(dt) or not a.flags.c_contiguous:
+            raise ValueError(f"output array {a.shape} {a.dtype} does not match {tuple(shape)} {dt}")
+    return out
+
+
+def gate_topk(logits, bias, k, score_fn, renormalize=True, out=None):
     logits = _c(logits, np.float32)
     T, E = logits.shape
     b = _c(bias, np.float32) if bias is not None else None
-    idx = np.empty((T, k), dtype=np.int32)
-    w = np.empty((T, k), dtype=np.float32)
+    idx, w = _outputs(out, ((T, k), np.int32), ((T, k), np.float32))
     rc = lib().tko_gate_topk(_p(logits), _p(b), T, E, k, score_fn, int(bool(renormalize)),
                              _p(idx), _p(w))
     if rc < 0:
@@ -123,13 +135,12 @@ def gate_topk(logits, bias, k, score_fn, renormalize=True):
     return idx, w
 
 
-def route_map(topk_idx, E, align=1):
+def route_map(topk_idx, E, align=1, out=None):
     topk_idx = _c(topk_idx, np.int32)
     T, k = topk_idx.shape
-    counts = np.empty(E, dtype=np.int32)
-    offsets = np.empty(E + 1, dtype=np.int32)
-    slot_of = np.empty((T, k), dtype=np.int32)
-    token_of = np.empty(max_rows(T, E, k, align), dtype=np.int32)
+    counts, offsets, slot_of, token_of = _outputs(
+        out, ((E,), np.int32), ((E + 1,), np.int32), ((T, k), np.int32),
+        ((max_rows(T, E, k, align),), np.int32))
     rc = lib().tko_route_map(_p(topk_idx), T, E, k, align, _p(counts), _p(offsets), _p(slot_of),
                              _p(token_of))
     if rc < 0:
@@ -147,16 +158,23 @@ def quantize_row_e4m3(xrow_bits):
     return q, s
 
 
-def expand(x_bits, slot_of, offsets, E, align=1, out_dtype=OUT_BF16):
+def expand(x_bits, slot_of, offsets, E, align=1, out_dtype=OUT_BF16, out=None):
     """Returns (out, out_scale); out has max_rows(T, E, k, align) rows, rows past offsets[E]
-    are left as zero here (the oracle never writes them)."""
+    are left as zero here (the oracle never writes them; caller-given arrays keep what they
+    held there)."""
     x_bits = _c(x_bits, np.uint16)
     slot_of = _c(slot_of, np.int32)
     offsets = _c(offsets, np.int32)
     T, H = x_bits.shape
     k = slot_of.shape[1]
     rmax = max_rows(T, E, k, align)
-    if out_dtype == OUT_BF16:
+    if out is not None:
+        if out_dtype == OUT_BF16:
+            (out,) = _outputs(out[:1], ((rmax, H), np.uint16))
+            scale = None
+        else:
+            out, scale = _outputs(out, ((rmax, H), np.uint8), ((rmax, H // 128), np.float32))
+    elif out_dtype == OUT_BF16:
         out = np.zeros((rmax, H), dtype=np.uint16)
         scale = None
     else:
@@ -180,13 +198,13 @@ def reduce_token(y_bits, slot_row, w_row):
     return out
 
 
-def reduce(y_bits, slot_of, w):
+def reduce(y_bits, slot_of, w, out=None):
     y_bits = _c(y_bits, np.uint16)
     slot_of = _c(slot_of, np.int32)
     w = _c(w, np.float32) if w is not None else None
     T, k = slot_of.shape
     H = y_bits.shape[1]
-    out = np.empty((T, H), dtype=np.uint16)
+    (out,) = _outputs(None if out is None else (out,), ((T, H), np.uint16))
     rc = lib().tko_reduce(_p(y_bits), y_bits.shape[0], _p(slot_of), _p(w), T, k, H, _p(out))
     if rc < 0:
         raise ValueError(f"tko_reduce rejected its arguments (rc={rc})")
