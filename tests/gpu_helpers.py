@@ -51,3 +51,14 @@ def assert_weights_close(w_gpu, w_ref, rtol=1e-6):
     err = np.abs(w_gpu - w_ref)
     bad = err > rtol * np.abs(w_ref)
     assert not bad.any(), f"{bad.sum()} weights off by more than {rtol} relative; worst {err.max()}"
+
+
+def assert_weights_round_alike(w_gpu, w_ref, max_share=1e-5):
+    """Both sides compute the weights in fp64 and round once to fp32, so they round alike: at
+    most a share `max_share` of them (and at least one allowed) may differ, by one fp32 ulp."""
+    a = np.ascontiguousarray(w_gpu, np.float32).view(np.int32).astype(np.int64)
+    b = np.ascontiguousarray(w_ref, np.float32).view(np.int32).astype(np.int64)
+    diff = np.abs(a - b)
+    n_diff = int((diff != 0).sum())
+    assert n_diff <= max(1, int(max_share * diff.size)), f"{n_diff} of {diff.size} weights differ"
+    assert diff.max(initial=0) <= 1, f"a weight differs by {diff.max()} fp32 ulps"

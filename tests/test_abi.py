@@ -41,8 +41,10 @@ def test_library_exports_every_declared_symbol(tk):
 def test_sizes_and_strings(tk):
     assert tk.max_rows(8192, 256, 8, 1) == 65536
     assert tk.max_rows(16384, 256, 8, 128) == 16384 * 8 + 256 * 127
-    assert tk.route_map_workspace_bytes(8192, 256, 8) == 32 * 256 * 4
-    assert tk.route_map_workspace_bytes(0, 16, 2) == 16 * 4
+    # E rows of per-tile counts, tiles of 128 tokens, each row padded to a multiple of 4 tiles
+    assert tk.route_map_workspace_bytes(8192, 256, 8) == 64 * 256 * 4
+    assert tk.route_map_workspace_bytes(8193, 256, 8) == 68 * 256 * 4
+    assert tk.route_map_workspace_bytes(0, 16, 2) == 4 * 16 * 4
     assert tk.lib.tk_status_str(0) == b"TK_OK"
     assert tk.lib.tk_status_str(1) == b"TK_ERR_INVALID_ARG"
     assert tk.lib.tk_abi_version() >> 16 == 1
