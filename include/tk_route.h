@@ -124,12 +124,13 @@ TK_API tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int 
  * owns all device memory and hands a component only its inputs and outputs, or a
  * latency-critical loop that must not call cudaMalloc, which can synchronise the device).
  * Same arguments, results and errors as tk_route_map, without workspace: the scratch it needs
- * is a 1 MiB array built into the library (every GPU that loads the library holds it until
- * the process exits). It serves T and E with ceil(T/256) * E <= 262144 (e.g. T <= 262144 at
- * E = 256, T <= 65536 at E = 1024); larger sizes return TK_ERR_INVALID_ARG and enqueue
- * nothing. The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current and caches it; make that first call before
- * any stream capture. All calls on a device share the array and nothing in it needs to start
+ * is a 2 MiB array built into the library (every GPU that loads the library holds it until
+ * the process exits). It serves T and E with E * 4*ceil(ceil(T/128)/4) <= 524288 (e.g.
+ * T <= 262144 at E = 256, T <= 65536 at E = 1024); larger sizes return TK_ERR_INVALID_ARG and
+ * enqueue nothing. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it for the life of the process;
+ * make that first call before any stream capture. A device reset (cudaDeviceReset) after the
+ * first call on that device is not supported: the cached address would be stale. All calls on a device share the array and nothing in it needs to start
  * at zero; calls that can overlap on the GPU (other streams, other host threads) race on it
  * and must be serialised by the caller. The call allocates nothing.
  */
@@ -352,6 +353,16 @@ TK_API tk_status tk_ep_combine(const void* const* partial, const int64_t* base_r
  * int32) and the kernel returns, leaving the context usable.
  */
 TK_API tk_status tk_selftest_bounded_wait(int64_t limit_ns, int32_t* err_flag, void* stream);
+
+/*
+ * Self-test of the gate's candidate filter (no counterpart on the pages: it checks on the GPU
+ * the error bound the filter's margin rests on). For every finite fp32 logit l with
+ * |l| <= 2^7 (about 2.2e9 values), the absolute difference between the filter's approximate
+ * logistic value (ex2.approx / rcp.approx) and the exact fp32 sigmoid of the selection key;
+ * the largest one is written to *max_err (device float; set to 0 first by this call). The
+ * filter assumes it is below 2^-17 and keeps a margin of 2^-12.
+ */
+TK_API tk_status tk_selftest_gate_margin(float* max_err, void* stream);
 
 /* Name of a status code (static string). */
 TK_API const char* tk_status_str(int status);

@@ -1,6 +1,5 @@
-// Per-token gate arithmetic shared by the gate kernel and the fused gate + route-map kernel
-// (one warp per token; lane l holds experts l, l+32, l+64, ...). See gate_topk.cu for the
-// method and its sources.
+// Per-token gate arithmetic of the gate kernel (one warp per token; lane l holds experts l,
+// l+32, l+64, ...). See gate_topk.cu for the method and its sources.
 #pragma once
 
 #include <math.h>
@@ -41,6 +40,55 @@ __device__ __forceinline__ float key_sigmoidf(float l) {
     return __fdiv_rn(1.0f, __fadd_rn(1.0f, key_expf(-l)));
 }
 
+// ---- fp64 arithmetic of the sigmoid weights. A weight only has to come within a few fp64 ulps
+// of s_j / sum(s) before it is rounded to fp32 (it then rounds like the oracle's fp64 value
+// except with probability ~2^-27), so these need not be correctly rounded.
+
+// e^x in fp64: Cody-Waite reduction by ln 2 (ln 2 split into a 21-bit high part, so n * hi is
+// exact for |n| < 2^11, and the fp64 remainder), degree-13 Taylor polynomial of e^r on
+// |r| <= ln2/2 (truncation below 6e-18) with coefficients 1/i! rounded to fp64, Horner with
+// fma, then 2^n in two exact steps. e^x overflows to +inf above ln(DBL_MAX) and is 0 below
+// -746, as a correctly rounded exponential does; NaN passes through.
+__device__ __forceinline__ double weight_exp(double x) {
+    if (x != x) return x;
+    if (x > 709.782712893384) return INFINITY;
+    if (x < -746.0) return 0.0;
+    const double n = rint(x * 0x1.71547652b82fep+0);
+    double r = fma(-n, 0x1.62e42p-1, x);
+    r = fma(-n, 0x1.fdf473de6af28p-22, r);
+    double p = 0x1.6124613a86d09p-33;     // 1/13!
+    p = fma(p, r, 0x1.1eed8eff8d898p-29);  // 1/12!
+    p = fma(p, r, 0x1.ae64567f544e4p-26);  // 1/11!
+    p = fma(p, r, 0x1.27e4fb7789f5cp-22);  // 1/10!
+    p = fma(p, r, 0x1.71de3a556c734p-19);  // 1/9!
+    p = fma(p, r, 0x1.a01a01a01a01ap-16);  // 1/8!
+    p = fma(p, r, 0x1.a01a01a01a01ap-13);  // 1/7!
+    p = fma(p, r, 0x1.6c16c16c16c17p-10);  // 1/6!
+    p = fma(p, r, 0x1.1111111111111p-7);   // 1/5!
+    p = fma(p, r, 0x1.5555555555555p-5);   // 1/4!
+    p = fma(p, r, 0x1.5555555555555p-3);   // 1/3!
+    p = fma(p, r, 0.5);
+    p = fma(p, r, 1.0);
+    p = fma(p, r, 1.0);
+    const int ni = static_cast<int>(n);    // [-1077, 1024]
+    const int n1 = ni / 2;
+    const int n2 = ni - n1;
+    return p * __hiloint2double((n1 + 1023) << 20, 0) * __hiloint2double((n2 + 1023) << 20, 0);
+}
+
+// 1/x in fp64 for x >= 2^-1000: the hardware's approximate reciprocal refined by two Newton
+// steps y += y (1 - x y) (each squares the relative error); IEEE division for huge or
+// infinite x.
+__device__ __forceinline__ double weight_rcp(double x) {
+    if (!(x < 0x1p+1000)) return 1.0 / x;
+    double y;
+    asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(x));
+    double e = fma(-x, y, 1.0);
+    y = fma(y, e, y);
+    e = fma(-x, y, 1.0);
+    return fma(y, e, y);
+}
+
 // Order-preserving map of an fp32 key to uint32 (larger key -> larger integer). -0 is folded
 // onto +0 and NaN onto -inf first, so float equality and integer equality agree.
 __device__ __forceinline__ uint32_t ordered_key(float key) {
@@ -76,6 +124,123 @@ __device__ __forceinline__ void sort_desc(uint64_t (&v)[EPL]) {
             }
         }
     }
+}
+
+// Inverse of ordered_key for the image of a real key (any value >= the image of -inf).
+__device__ __forceinline__ float key_of_image(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// Hardware approximations for the candidate filter only (no result is taken from them).
+// PTX ISA: rcp.approx.f32 is within 1 ulp; ex2.approx.f32 within a few ulp (relative error
+// about 2^-22); .ftz flushes subnormal results to zero.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Approximate logistic value 1 / (1 + 2^(-l log2 e)). Rounding l log2 e to fp32 moves the
+// exponent by at most |l| log2 e 2^-24, a relative error of at most 6e-6 in 2^x for
+// |l| <= 100; with the approximations' own errors the value is within 2^-17 of the true
+// logistic value there (its slope in log e^-l is s(1-s) <= 1/4), as is the exact key's fp32
+// sigmoid (within 2^-22). Beyond |l| = 100 both are 0 or 1 to within 2^-126.
+__device__ __forceinline__ float approx_sigmoidf(float l) {
+    return rcp_approx(1.0f + ex2_approx(l * -0x1.715476p+0f));
+}
+
+// Order-preserving image of an approximate key: NaN ranks as -inf (fmaxf keeps the other
+// operand), so a NaN logit sorts at the bottom exactly as its exact key does.
+__device__ __forceinline__ uint32_t approx_image(float a) {
+    a = fmaxf(a, -INFINITY);
+    const uint32_t u = __float_as_uint(a);
+    return u ^ ((static_cast<uint32_t>(static_cast<int32_t>(u) >> 31)) | 0x80000000u);
+}
+
+// Images of the lane's approximate keys (0 for an absent expert e >= E). Without a bias the
+// key is the logit itself (-0 folded onto +0 like the exact key), so the image is exact.
+template <int EPL>
+__device__ __forceinline__ void approx_images(const float (&lg)[EPL], const float (&b)[EPL],
+                                              bool has_bias, int E, int lane, uint32_t (&u)[EPL]) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        const float a = has_bias ? __fadd_rn(approx_sigmoidf(lg[i]), b[i]) : __fadd_rn(lg[i], 0.0f);
+        u[i] = e < E ? approx_image(a) : 0u;
+    }
+}
+
+// A value with at least k of the 32 lanes' values >= it, cheaply: with G = the smallest power
+// of two >= k, the minimum over G groups of 32/G adjacent lanes of each group's maximum (each
+// group contributes one value >= it). 0 when some group holds no expert.
+__device__ __forceinline__ uint32_t group_threshold(uint32_t v, int k) {
+    int width = 32;  // lanes per group
+    while (width > 1 && 32 / width < k) width >>= 1;
+    for (int off = 1; off < width; off <<= 1) v = max(v, __shfl_xor_sync(kFullMask, v, off));
+    for (int off = width; off < 32; off <<= 1) v = min(v, __shfl_xor_sync(kFullMask, v, off));
+    return v;
+}
+
+// The k-th largest of the 32 lanes' values, counted with multiplicity: at least k lanes hold a
+// value >= the result. 0 when fewer than k lanes hold a nonzero value. Warp-uniform.
+__device__ __forceinline__ uint32_t kth_lane_max(uint32_t v, int k) {
+    int have = 0;
+    for (int r = 0; r < k; ++r) {
+        const uint32_t m = __reduce_max_sync(kFullMask, v);
+        if (m == 0) return 0;
+        have += __popc(__ballot_sync(kFullMask, v == m));
+        if (have >= k) return m;
+        if (v == m) v = 0;
+    }
+    return 0;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// One warp's shared scratch: the candidates (expert, logit bits) in (slot of the lane's list,
+// lane) order, and the chosen experts by rank.
+struct Candidates {
+    uint2 el[32];
+    int by_rank[32];
+};
+
+// Ballots of the lane's experts whose image is >= cut; returns their number (warp-uniform).
+template <int EPL>
+__device__ __forceinline__ int count_candidates(const uint32_t (&u)[EPL], uint32_t cut,
+                                                uint32_t (&bal)[EPL]) {
+    int C = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        bal[i] = __ballot_sync(kFullMask, u[i] >= cut);
+        C += __popc(bal[i]);
+    }
+    return C;
+}
+
+// Writes the balloted candidates (at most 32) to the warp's list, candidate c at entry c.
+template <int EPL>
+__device__ __forceinline__ void gather_candidates(const uint32_t (&bal)[EPL], const float (&lg)[EPL],
+                                                  int lane, Candidates& c) {
+    const uint32_t lt = lanemask_lt();
+    int base = 0;
+    __syncwarp();  // the previous token's reads of the list are done
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        if ((bal[i] >> lane) & 1u)
+            c.el[base + __popc(bal[i] & lt)] = make_uint2(static_cast<uint32_t>(i * 32 + lane),
+                                                          __float_as_uint(lg[i]));
+        base += __popc(bal[i]);
+    }
+    __syncwarp();
 }
 
 // Keys of the lane's experts, packed with their indices (0 for an absent expert e >= E). Every

@@ -26,15 +26,67 @@ namespace {
 
 constexpr int kGateWarps = 8;  // tokens per CTA
 
+// Selection in two passes, with the same result as ranking all E exact keys:
+//  1. Approximate keys A_e (the logit itself without a bias; approx_sigmoidf(l) + b with one)
+//     satisfy |A_e - K_e| <= eps for the exact keys K_e, where eps = 2^-12 + 2^-20 * max|b|
+//     is more than 30 times the bound in approx_sigmoidf's comment (the two additions of b
+//     round by at most an ulp of 1 + max|b| between them). Without a bias eps = 0.
+//  2. A threshold theta that at least k approximate keys reach (first the cheap
+//     group_threshold, then the k-th largest lane maximum when the cheap one leaves more than
+//     32 candidates). The k-th largest exact key is then >= theta - eps, and every expert whose
+//     exact key reaches it has A >= theta - 2 eps. Those experts (the candidates) get their
+//     exact keys, one per lane, and k rounds of two warp reductions select among them exactly
+//     as among all E; each winner keeps its rank and writes its own outputs.
+// More than 32 candidates (many equal or nearly equal keys), a non-finite or huge bias, or
+// fewer than k lanes holding an expert send the token down the full path: every exact key, a
+// per-lane sort and k rounds over the sorted lists.
+//
+// Weights are computed in fp64 and rounded once to fp32, as in the oracle: fp32 weights
+// within the 1e-6 bar but a few ulps off the oracle's would move reduce outputs that nearly
+// cancel by more than one bf16 ulp.
+__device__ __forceinline__ float filter_margin(const float* b, int epl, bool has_bias, bool* ok) {
+    if (!has_bias) {
+        *ok = true;
+        return 0.0f;
+    }
+    float m = 0.0f;
+    bool finite = true;
+    for (int i = 0; i < epl; ++i) {
+        finite = finite && isfinite(b[i]);
+        m = fmaxf(m, fabsf(b[i]));
+    }
+    finite = __all_sync(kFullMask, finite);
+    // |b| of finite values are non-negative floats: their bit patterns order like the values
+    m = __uint_as_float(__reduce_max_sync(kFullMask, __float_as_uint(finite ? m : 0.0f)));
+    *ok = finite && m < 0x1p+20f;
+    return __fmaf_ru(m, 0x1p-20f, 0x1p-12f);
+}
+
+// Candidate cut for a threshold image: theta itself without a bias, else the image of
+// theta - 2 eps rounded down.
+__device__ __forceinline__ uint32_t cut_of(uint32_t theta, bool has_bias, float eps) {
+    return has_bias ? gate::ordered_key(__fsub_rd(gate::key_of_image(theta), 2.0f * eps)) : theta;
+}
+
+template <int EPL>
+__device__ __forceinline__ void prefetch_row(const float* row, int E, int lane, float (&lg)[EPL]) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        lg[i] = e < E ? row[e] : 0.0f;
+    }
+}
+
 // One warp per token. The grid is one wave of resident warps and the T tokens are split evenly
 // over the nwarps warps (warp w takes tokens [w*T/nwarps, (w+1)*T/nwarps), so warps differ by
 // at most one token and every SM gets the same work); the next token's logits are loaded while
 // the current one is processed. EPL = experts held per lane (E <= 32 * EPL).
 template <int EPL>
-__global__ void __launch_bounds__(kGateWarps * 32)
+__global__ void __launch_bounds__(kGateWarps * 32, EPL <= 8 ? 4 : 1)
 gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                  int k, int score_fn, int renormalize, int nwarps,
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    __shared__ gate::Candidates cands[kGateWarps];
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t wid = static_cast<int64_t>(blockIdx.x) * kGateWarps + (threadIdx.x >> 5);
@@ -42,13 +94,18 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
     const int64_t t_begin = wid * T / nwarps;
     const int64_t t_end = (wid + 1) * T / nwarps;
     if (t_begin >= t_end) return;
+    gate::Candidates& cand = cands[threadIdx.x >> 5];
+    const bool has_bias = bias != nullptr;
+    const bool sigmoid = score_fn == TK_SCORE_SIGMOID;
 
     float b[EPL];  // this lane's selection biases, shared by all tokens
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = i * 32 + lane;
-        b[i] = (bias != nullptr && e < E) ? bias[e] : 0.0f;
+        b[i] = (has_bias && e < E) ? bias[e] : 0.0f;
     }
+    bool can_filter;
+    const float eps = filter_margin(b, EPL, has_bias, &can_filter);
     float lg[EPL];  // logits of the token being routed, then of the next one (prefetch)
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
@@ -58,18 +115,79 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
 
     for (int64_t t = t_begin; t < t_end; ++t) {
         const float* row = logits + t * E;
-        uint64_t v[EPL];
-        gate::build_keys<EPL>(lg, b, bias != nullptr, E, lane, v);
-        if (t + 1 < t_end) {  // the registers are free again: start the next token's loads
+        int32_t* idx_out = topk_idx + t * k;
+        float* w_out = topk_w + t * k;
+        int C = 33;  // > 32: full path
+        if (can_filter) {
+            uint32_t u[EPL], bal[EPL];
+            gate::approx_images<EPL>(lg, b, has_bias, E, lane, u);
+            uint32_t lane_max = u[0];
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int e = i * 32 + lane;
-                lg[i] = e < E ? row[E + e] : 0.0f;
+            for (int i = 1; i < EPL; ++i) lane_max = max(lane_max, u[i]);
+            uint32_t theta = gate::group_threshold(lane_max, k);
+            if (theta != 0) C = gate::count_candidates<EPL>(u, cut_of(theta, has_bias, eps), bal);
+            if (C > 32) {
+                theta = gate::kth_lane_max(lane_max, k);
+                if (theta != 0) C = gate::count_candidates<EPL>(u, cut_of(theta, has_bias, eps), bal);
+            }
+            if (C <= 32) gate::gather_candidates<EPL>(bal, lg, lane, cand);
+        }
+        if (C > 32) {  // full path (the current logits are still in lg)
+            uint64_t v[EPL];
+            gate::build_keys<EPL>(lg, b, has_bias, E, lane, v);
+            if (t + 1 < t_end) prefetch_row<EPL>(row + E, E, lane, lg);
+            const int my_e = gate::select_topk<EPL>(v, k, lane);
+            gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, idx_out, w_out);
+            continue;
+        }
+        // the candidates are captured: start the next token's loads
+        if (t + 1 < t_end) prefetch_row<EPL>(row + E, E, lane, lg);
+        // exact keys of the candidates, one per lane
+        int e = 0;
+        float l = 0.0f;
+        uint32_t hi = 0, lo = 0;
+        if (lane < C) {
+            const uint2 el = cand.el[lane];
+            e = static_cast<int>(el.x);
+            l = __uint_as_float(el.y);
+            const float key = has_bias ? __fadd_rn(gate::key_sigmoidf(l), __ldg(bias + e)) : l;
+            hi = gate::ordered_key(key);
+            lo = ~static_cast<uint32_t>(e);
+        }
+        // k rounds: the largest key, ties to the lower expert index; the winner keeps its rank
+        int rank = k;
+        for (int j = 0; j < k; ++j) {
+            const uint32_t m = __reduce_max_sync(kFullMask, hi);
+            const uint32_t win = __reduce_max_sync(kFullMask, hi == m ? lo : 0u);
+            if (hi == m && lo == win) {
+                rank = j;
+                hi = 0;
             }
         }
-        const int my_e = gate::select_topk<EPL>(v, k, lane);
-        gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, topk_idx + t * k,
-                                topk_w + t * k);
+        const bool chosen = rank < k;
+        if (!sigmoid) {  // softmax weights need the whole row: lane j takes the j-th expert
+            if (chosen) cand.by_rank[rank] = e;
+            __syncwarp();
+            const int my_e = lane < k ? cand.by_rank[lane] : 0;
+            gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, idx_out, w_out);
+            continue;
+        }
+        // weights in fp64 (within a few fp64 ulps of the exact value), rounded once to fp32, so
+        // they round like the oracle's and the reduce that uses them agrees with it too
+        const double sd = chosen ? gate::weight_rcp(1.0 + gate::weight_exp(-static_cast<double>(l))) : 0.0;
+        double denom = sd;
+        if (renormalize) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) denom += __shfl_xor_sync(kFullMask, denom, off);
+        }
+        if (chosen) {
+            float w = static_cast<float>(sd);
+            if (renormalize)
+                w = denom == 0.0 ? 0.0f
+                    : static_cast<float>(denom >= 0x1p-1000 ? sd * gate::weight_rcp(denom) : sd / denom);
+            idx_out[rank] = e;
+            w_out[rank] = w;
+        }
     }
 }
 
@@ -94,8 +212,35 @@ cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, in
                       k, score_fn, renormalize, warps, idx, w);
 }
 
+// Largest |approx_sigmoidf(l) - key_sigmoidf(l)| over the finite fp32 l with |l| <= 2^7: the
+// positive-and-negative bit patterns below 0x43000001 (2^7), grid-stride.
+__global__ void __launch_bounds__(256) gate_margin_kernel(uint32_t* max_err_bits) {
+    constexpr uint32_t kLimit = 0x43000001u;  // bit patterns of [0, 2^7]
+    uint32_t worst = 0;
+    const uint64_t n = 2ull * kLimit;
+    for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+        const uint32_t mag = static_cast<uint32_t>(i >> 1);
+        const float l = __uint_as_float(mag | (static_cast<uint32_t>(i & 1) << 31));
+        const float d = fabsf(gate::approx_sigmoidf(l) - gate::key_sigmoidf(l));
+        worst = max(worst, __float_as_uint(d));  // non-negative floats order like their bits
+    }
+    worst = __reduce_max_sync(kFullMask, worst);
+    if ((threadIdx.x & 31) == 0) atomicMax(max_err_bits, worst);
+}
+
 }  // namespace
 }  // namespace tk
+
+extern "C" tk_status tk_selftest_gate_margin(float* max_err, void* stream) {
+    using namespace tk;
+    if (max_err == nullptr) return fail_arg("tk_selftest_gate_margin: max_err must not be NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaMemsetAsync(max_err, 0, sizeof(float), s);
+    if (err != cudaSuccess) return check_launch(err, "tk_selftest_gate_margin: cudaMemsetAsync");
+    gate_margin_kernel<<<num_sms() * 8, 256, 0, s>>>(reinterpret_cast<uint32_t*>(max_err));
+    return check_launch(cudaGetLastError(), "gate_margin_kernel");
+}
 
 extern "C" tk_status tk_gate_topk(const float* logits, const float* bias, int T, int E, int k,
                                   int score_fn, int renormalize, int32_t* topk_idx, float* topk_w,

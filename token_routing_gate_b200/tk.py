@@ -34,6 +34,7 @@ ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "t
                "tk_balance_stats", "tk_balance_score_sums", "tk_balance_finalize", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
                "tk_reduce_backward", "tk_expand_backward", "tk_ep_layout_workspace_bytes",
                "tk_ep_layout", "tk_ep_dispatch", "tk_ep_combine", "tk_selftest_bounded_wait",
+               "tk_selftest_gate_margin",
                "tk_status_str", "tk_last_error_detail", "tk_abi_version")
 
 
@@ -102,6 +103,8 @@ def _load():
     L.tk_ep_combine.restype = i32
     L.tk_selftest_bounded_wait.argtypes = [i64, vp, vp]
     L.tk_selftest_bounded_wait.restype = i32
+    L.tk_selftest_gate_margin.argtypes = [vp, vp]
+    L.tk_selftest_gate_margin.restype = i32
     L.tk_status_str.argtypes = [i32]
     L.tk_status_str.restype = ctypes.c_char_p
     L.tk_last_error_detail.argtypes = []
@@ -349,6 +352,16 @@ def selftest_bounded_wait(limit_ns, err_flag, stream=None):
     """Run the bounded-wait self-test kernel (it always times out and flags DEVERR_TIMEOUT)."""
     _check("tk_selftest_bounded_wait", lib.tk_selftest_bounded_wait(int(limit_ns), _flag(err_flag),
                                                                     _stream(stream)))
+
+
+def selftest_gate_margin(max_err=None, stream=None):
+    """Largest |approximate - exact| logistic value over the finite fp32 logits |l| <= 2^7 (the
+    bound the gate's candidate filter rests on), as a device float tensor [1]."""
+    if max_err is None:
+        max_err = torch.empty(1, dtype=torch.float32, device="cuda")
+    _check("tk_selftest_gate_margin", lib.tk_selftest_gate_margin(_ptr(max_err, F32, 1, "max_err"),
+                                                                  _stream(stream)))
+    return max_err
 
 
 # ---------------------------------------------------------------- expert-parallel dispatch / combine
