@@ -365,8 +365,10 @@ def run_tk(args, wl):
         if ev is not None:
             ev[4].record(stream)
 
-    tiles = (wl.T + 255) // 256                  # route map: count + fused scan/scatter up to
-    route_launches = 2 if tiles <= 128 else 3    # 128 tiles of 256 tokens, else three kernels
+    # route map: count + fused scan/scatter while its count matrix (E rows of 128-token tiles,
+    # padded to a multiple of 4) has at most 64K entries, else count, scan and scatter
+    tiles = (wl.T + 127) // 128
+    route_launches = 2 if (tiles + 3) // 4 * 4 * wl.E <= 65536 else 3
     launches_per_step = 1 + route_launches + 1 + (1 if wl.align > 1 else 0) + 1
     for _ in range(args.warmup):
         step()

@@ -3,13 +3,13 @@
 // mapping is one of the MoE routing ops).
 //
 // The pairs p = t*k + j are cut into tiles of kTileTokens tokens. Three short kernels (the last
-// two run as one kernel, route_scan_scatter_kernel, while the batch has at most 128 tiles):
+// two run as one kernel, route_scan_scatter_kernel, while the count matrix is small):
 //   count   : one CTA per tile counts its pairs per expert in shared memory (integer atomics,
-//             so the counts do not depend on their order) and writes a row of the
-//             [tiles x E] count matrix; the grid also fills token_of with -1.
-//   scan    : one CTA turns each column of the matrix into exclusive per-tile prefixes, sums
-//             the column into counts[e], rounds it up to the alignment and scans over experts
-//             for offsets[].
+//             so the counts do not depend on their order) and writes a column of the
+//             [E x tiles] count matrix (expert-major, each expert's row padded to a multiple of
+//             4 tiles so that it reads as 16-byte vectors); the grid also fills token_of with -1.
+//   scan    : turns each expert's row into exclusive per-tile prefixes, sums it into
+//             counts[e], rounds it up to the alignment and scans over experts for offsets[].
 //   scatter : one CTA per tile marks, per expert, which of its tokens chose that expert in a
 //             shared-memory bitmap; a pair's rank inside the tile is the population count of
 //             the bits below its token. slot = offsets[e] + tile prefix[e] + rank -- the same
@@ -23,15 +23,19 @@
 namespace tk {
 namespace {
 
-constexpr int kTileTokens = 256;               // tokens per tile
+constexpr int kTileTokens = 128;               // tokens per tile
 constexpr int kTileWords = kTileTokens / 32;   // bitmap words per expert
 constexpr int kRouteThreads = 512;
-constexpr int kPairsPerThread = kTileTokens * TK_MAX_TOPK / kRouteThreads;  // 16
+constexpr int kPairsPerThread = kTileTokens * TK_MAX_TOPK / kRouteThreads;  // 8
 constexpr int kScanThreads = 1024;
-constexpr int kScanBatch = 32;                 // column loads in flight per thread
-constexpr int kFusedMaxTiles = 128;            // up to here every scatter CTA scans for itself
+constexpr int kRowBatch = 8;                   // 16-byte loads in flight per expert row
+// The fused scan + scatter kernel has every CTA read the whole count matrix; beyond this many
+// entries the separate scan kernel reads it once instead.
+constexpr int64_t kFusedMaxEntries = 64 * 1024;
 
 inline int num_tiles(int T) { return (T + kTileTokens - 1) / kTileTokens; }
+// Row length of the count matrix: the tiles rounded up to whole 16-byte vectors.
+inline int row_stride(int tiles) { return (tiles + 3) / 4 * 4; }
 
 // The scan kernel gives each expert its own thread: E rounded up to whole warps.
 inline int scan_threads(int E) {
@@ -39,22 +43,39 @@ inline int scan_threads(int E) {
     return t < kScanThreads ? t : kScanThreads;
 }
 
+// Exact n / k for 0 <= n < 2^16 and 1 <= k <= 32 by a multiply-high with m = ceil(2^32 / k):
+// n * m / 2^32 = n / k + n * r / (k * 2^32) with r = m*k - 2^32 < k, and the second term is
+// below 2^-16 / k, too small to carry n / k past the next integer.
+struct DivK {
+    uint64_t m;
+    __device__ __forceinline__ explicit DivK(int k)
+        : m((UINT64_C(0x100000000) + static_cast<uint64_t>(k) - 1) / static_cast<uint64_t>(k)) {}
+    __device__ __forceinline__ int operator()(int n) const {
+        return static_cast<int>((static_cast<uint64_t>(n) * m) >> 32);
+    }
+};
+
+// Pairs p0 + threadIdx.x + i * kRouteThreads, i < the result, lie inside a tile of n pairs.
+__device__ __forceinline__ int pairs_of_thread(int n) {
+    return n > static_cast<int>(threadIdx.x) ? (n - 1 - static_cast<int>(threadIdx.x)) / kRouteThreads + 1 : 0;
+}
+
 __global__ void __launch_bounds__(kRouteThreads)
 route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                   int32_t* __restrict__ tile_counts, int32_t* __restrict__ token_of,
+                   int32_t* __restrict__ tile_counts, int stride, int32_t* __restrict__ token_of,
                    int64_t rmax, int32_t* err_flag) {
     extern __shared__ int32_t cnt[];  // [E]
     pdl_wait();
     const int tile = blockIdx.x;
     const int64_t p0 = static_cast<int64_t>(tile) * kTileTokens * k;
-    const int64_t p1 = min(static_cast<int64_t>(T), static_cast<int64_t>(tile + 1) * kTileTokens) * k;
+    const int n = static_cast<int>(min(static_cast<int64_t>(T), static_cast<int64_t>(tile + 1) * kTileTokens) * k - p0);
     // all index loads of this thread first, so their latencies overlap
-    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
     int e_reg[kPairsPerThread];
+    const int mine = pairs_of_thread(n);
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
+        if (i >= mine) break;
+        e_reg[i] = topk_idx[p0 + threadIdx.x + i * kRouteThreads];
     }
     for (int e = threadIdx.x; e < E; e += kRouteThreads) cnt[e] = 0;
     // every row starts as "no token"; the scatter kernel fills the real rows afterwards
@@ -64,9 +85,7 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        if (p >= p1) continue;
+        if (i >= mine) break;
         const int e = e_reg[i];
         if (e < 0 || e >= E) {  // -1 is a masked pair (tk_tp_mask), anything else an error
             if (e != -1) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
@@ -75,24 +94,30 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
         atomicAdd(&cnt[e], 1);  // integer counts: the order of the additions does not matter
     }
     __syncthreads();
-    if (p0 < p1 || tile == 0) {
+    if (n > 0) {
         for (int e = threadIdx.x; e < E; e += kRouteThreads)
-            tile_counts[static_cast<int64_t>(tile) * E + e] = cnt[e];
+            tile_counts[static_cast<int64_t>(e) * stride + tile] = cnt[e];
+    }
+    // the last tile also zeroes each row's padding, so rows can be summed in whole vectors
+    if (tile == gridDim.x - 1) {
+        const int pad = stride - (tile + 1);
+        for (int i = threadIdx.x; i < E * pad; i += kRouteThreads)
+            tile_counts[static_cast<int64_t>(i / pad) * stride + tile + 1 + i % pad] = 0;
     }
 }
 
 // ---- rank phase shared by every scatter variant: bitmap of the tile's tokens per expert, then
 // slot = base[e] + (number of the tile's earlier tokens on expert e)
 __device__ __forceinline__ void tile_mark(uint32_t* bitmap, const int (&e_reg)[kPairsPerThread],
-                                          int iters, int64_t p0, int64_t p1, int k, int t0, int E,
-                                          int32_t* err_flag) {
+                                          int n, const DivK& divk, int E, int32_t* err_flag) {
+    const int mine = pairs_of_thread(n);
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
+        if (i >= mine) break;
+        const int pl = threadIdx.x + i * kRouteThreads;
         const int e = e_reg[i];
-        if (p >= p1 || e < 0 || e >= E) continue;  // out-of-range experts: flagged elsewhere
-        const int tl = static_cast<int>(p / k) - t0;
+        if (e < 0 || e >= E) continue;  // out-of-range experts: flagged elsewhere
+        const int tl = divk(pl);
         const uint32_t bit = 1u << (tl & 31);
         const uint32_t old = atomicOr(&bitmap[e * kTileWords + (tl >> 5)], bit);
         if (old & bit) flag_error(err_flag, TK_DEVERR_DUP_EXPERT);
@@ -100,39 +125,87 @@ __device__ __forceinline__ void tile_mark(uint32_t* bitmap, const int (&e_reg)[k
 }
 
 __device__ __forceinline__ void tile_scatter(const uint32_t* bitmap, const int32_t* base,
-                                             const int (&e_reg)[kPairsPerThread], int iters,
-                                             int64_t p0, int64_t p1, int k, int t0, int E,
+                                             const int (&e_reg)[kPairsPerThread], int n,
+                                             const DivK& divk, int64_t p0, int t0, int E,
                                              int32_t* slot_of, int32_t* token_of) {
+    const int mine = pairs_of_thread(n);
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
-        if (i >= iters) break;
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        if (p >= p1) continue;
+        if (i >= mine) break;
+        const int pl = threadIdx.x + i * kRouteThreads;
         const int e = e_reg[i];
         if (e < 0 || e >= E) {
-            slot_of[p] = -1;
+            slot_of[p0 + pl] = -1;
             continue;
         }
-        const int t = static_cast<int>(p / k);
-        const int tl = t - t0;
+        const int tl = divk(pl);
         const uint32_t* bm = bitmap + e * kTileWords;
         int rank = __popc(bm[tl >> 5] & ((1u << (tl & 31)) - 1u));
-        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bm[w]);
+#pragma unroll
+        for (int w = 0; w + 1 < kTileWords; ++w)
+            if (w < (tl >> 5)) rank += __popc(bm[w]);
         const int32_t slot = base[e] + rank;
-        slot_of[p] = slot;
-        token_of[slot] = t;
+        slot_of[p0 + pl] = slot;
+        token_of[slot] = t0 + tl;
     }
 }
 
-__device__ __forceinline__ int load_tile(const int32_t* topk_idx, int64_t p0, int64_t p1,
-                                         int (&e_reg)[kPairsPerThread]) {
-    const int iters = static_cast<int>((p1 - p0 + kRouteThreads - 1) / kRouteThreads);
+__device__ __forceinline__ void load_tile(const int32_t* topk_idx, int64_t p0, int n,
+                                          int (&e_reg)[kPairsPerThread]) {
+    const int mine = pairs_of_thread(n);
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
-        const int64_t p = p0 + threadIdx.x + static_cast<int64_t>(i) * kRouteThreads;
-        e_reg[i] = (i < iters && p < p1) ? topk_idx[p] : -1;
+        if (i >= mine) break;
+        e_reg[i] = topk_idx[p0 + threadIdx.x + i * kRouteThreads];
     }
-    return iters;
+}
+
+// Sums of expert rows of the count matrix over the tiles before `tile` and over all tiles,
+// into before[e] and total[e]. P = 1, 2, 4 or 8 neighbouring threads share a row, each summing
+// every P-th 16-byte vector (kRowBatch loads in flight), then they add their sums. Padding
+// entries past the last tile are zero (written by the count kernel), so whole vectors are
+// summed; only the vector that holds `tile` is masked.
+__device__ __forceinline__ void row_sums(const int32_t* tile_counts, int stride, int E, int tile,
+                                         int32_t* before, int32_t* total) {
+    int P = 1;
+    while (P < 8 && P * 2 * E <= kRouteThreads) P *= 2;
+    const int part = threadIdx.x % P;
+    const int n4 = stride / 4;
+    const int rounds = (E * P + kRouteThreads - 1) / kRouteThreads;
+    for (int r = 0; r < rounds; ++r) {
+        const int e = (r * kRouteThreads + threadIdx.x) / P;
+        int32_t b = 0, tot = 0;
+        if (e < E) {
+            const int4* r4 = reinterpret_cast<const int4*>(tile_counts + static_cast<int64_t>(e) * stride);
+            for (int c0 = part; c0 < n4; c0 += P * kRowBatch) {
+                int4 v[kRowBatch];
+#pragma unroll
+                for (int i = 0; i < kRowBatch; ++i) {
+                    const int c4 = c0 + i * P;
+                    v[i] = c4 < n4 ? r4[c4] : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < kRowBatch; ++i) {
+                    const int c = (c0 + i * P) * 4;
+                    const int32_t s4 = v[i].x + v[i].y + v[i].z + v[i].w;
+                    tot += s4;
+                    if (c + 4 <= tile) {
+                        b += s4;
+                    } else if (c < tile) {
+                        b += v[i].x + (c + 1 < tile ? v[i].y : 0) + (c + 2 < tile ? v[i].z : 0);
+                    }
+                }
+            }
+        }
+        for (int off = 1; off < P; off <<= 1) {
+            b += __shfl_xor_sync(kFullMask, b, off);
+            tot += __shfl_xor_sync(kFullMask, tot, off);
+        }
+        if (e < E && part == 0) {
+            before[e] = b;
+            total[e] = tot;
+        }
+    }
 }
 
 // Exclusive scan of ceil(total[e]/align)*align over experts, for a whole CTA of kRouteThreads
@@ -171,9 +244,9 @@ __device__ __forceinline__ int32_t cta_padded_scan(const int32_t* total, int E, 
     return carry;
 }
 
-// Single CTA. Column e of tile_counts becomes exclusive per-tile prefixes (in place).
+// Single CTA. Each expert's row of tile_counts becomes exclusive per-tile prefixes (in place).
 __global__ void __launch_bounds__(kScanThreads)
-route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align,
+route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int stride, int E, int align,
                   int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
     __shared__ int32_t warp_tot[kScanThreads / 32];
     __shared__ int32_t carry;
@@ -187,16 +260,23 @@ route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align
         const int e = e0 + threadIdx.x;
         int32_t padded = 0;
         if (e < E) {
+            int4* r4 = reinterpret_cast<int4*>(tile_counts + static_cast<int64_t>(e) * stride);
+            const int n4 = (tiles + 3) / 4;
             int32_t run = 0;
-            for (int c0 = 0; c0 < tiles; c0 += kScanBatch) {
-                int32_t v[kScanBatch];
+            for (int c0 = 0; c0 < n4; c0 += kRowBatch) {
+                int4 v[kRowBatch];
 #pragma unroll
-                for (int i = 0; i < kScanBatch; ++i)
-                    v[i] = c0 + i < tiles ? tile_counts[static_cast<int64_t>(c0 + i) * E + e] : 0;
+                for (int i = 0; i < kRowBatch; ++i) v[i] = c0 + i < n4 ? r4[c0 + i] : make_int4(0, 0, 0, 0);
 #pragma unroll
-                for (int i = 0; i < kScanBatch; ++i) {
-                    if (c0 + i < tiles) tile_counts[static_cast<int64_t>(c0 + i) * E + e] = run;
-                    run += v[i];
+                for (int i = 0; i < kRowBatch; ++i) {
+                    if (c0 + i >= n4) break;
+                    const int c = (c0 + i) * 4;
+                    int4 o;
+                    o.x = run; run += c + 0 < tiles ? v[i].x : 0;
+                    o.y = run; run += c + 1 < tiles ? v[i].y : 0;
+                    o.z = run; run += c + 2 < tiles ? v[i].z : 0;
+                    o.w = run; run += c + 3 < tiles ? v[i].w : 0;
+                    r4[c0 + i] = o;
                 }
             }
             counts[e] = run;
@@ -235,9 +315,9 @@ route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int E, int align
 
 __global__ void __launch_bounds__(kRouteThreads)
 route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                     const int32_t* __restrict__ tile_prefix, const int32_t* __restrict__ offsets,
-                     int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
-                     int32_t* err_flag) {
+                     const int32_t* __restrict__ tile_prefix, int stride,
+                     const int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
+                     int32_t* __restrict__ token_of, int32_t* err_flag) {
     extern __shared__ uint32_t smem[];
     uint32_t* bitmap = smem;                                          // [E][kTileWords]
     int32_t* base = reinterpret_cast<int32_t*>(smem + E * kTileWords);  // [E]
@@ -245,25 +325,26 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     const int tile = blockIdx.x;
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
-    const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
+    const int n = (min(T, t0 + kTileTokens) - t0) * k;
+    const DivK divk(k);
     int e_reg[kPairsPerThread];
-    const int iters = load_tile(topk_idx, p0, p1, e_reg);
+    load_tile(topk_idx, p0, n, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     for (int e = threadIdx.x; e < E; e += kRouteThreads)
-        base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(tile) * E + e];
+        base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(e) * stride + tile];
     __syncthreads();
-    tile_mark(bitmap, e_reg, iters, p0, p1, k, t0, E, err_flag);
+    tile_mark(bitmap, e_reg, n, divk, E, err_flag);
     __syncthreads();
-    tile_scatter(bitmap, base, e_reg, iters, p0, p1, k, t0, E, slot_of, token_of);
+    tile_scatter(bitmap, base, e_reg, n, divk, p0, t0, E, slot_of, token_of);
 }
 
-// Scan and scatter in one kernel, for batches of at most kFusedMaxTiles tiles: every CTA reads
-// the whole (small) count matrix itself -- its own tile's prefix per expert, and every column's
-// total for the offsets -- instead of waiting for a separate scan kernel. CTA 0 also writes
-// counts[] and offsets[]. The slot arithmetic is the same as route_scan + route_scatter.
+// Scan and scatter in one kernel, for count matrices of at most kFusedMaxEntries entries: every
+// CTA reads the whole (small) count matrix itself -- its own tile's prefix per expert, and every
+// row's total for the offsets -- instead of waiting for a separate scan kernel. CTA 0 also
+// writes counts[] and offsets[]. The slot arithmetic is the same as route_scan + route_scatter.
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int align,
-                          const int32_t* __restrict__ tile_counts, int tiles,
+                          const int32_t* __restrict__ tile_counts, int stride,
                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                           int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
                           int32_t* err_flag) {
@@ -277,27 +358,13 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
     const int tile = blockIdx.x;
     const int t0 = tile * kTileTokens;
     const int64_t p0 = static_cast<int64_t>(t0) * k;
-    const int64_t p1 = static_cast<int64_t>(min(T, t0 + kTileTokens)) * k;
+    const int n = (min(T, t0 + kTileTokens) - t0) * k;
+    const DivK divk(k);
     int e_reg[kPairsPerThread];
-    const int iters = load_tile(topk_idx, p0, p1, e_reg);
+    load_tile(topk_idx, p0, n, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
-    // per expert: the count over the tiles before this one, and the column total
-    for (int e = threadIdx.x; e < E; e += kRouteThreads) {
-        int32_t b = 0, tot = 0;
-        for (int c0 = 0; c0 < tiles; c0 += kScanBatch) {
-            int32_t v[kScanBatch];
-#pragma unroll
-            for (int i = 0; i < kScanBatch; ++i)
-                v[i] = c0 + i < tiles ? tile_counts[static_cast<int64_t>(c0 + i) * E + e] : 0;
-#pragma unroll
-            for (int i = 0; i < kScanBatch; ++i) {
-                if (c0 + i < tile) b += v[i];
-                tot += v[i];
-            }
-        }
-        before[e] = b;
-        total[e] = tot;
-    }
+    // per expert: the count over the tiles before this one, and the row total
+    row_sums(tile_counts, stride, E, tile, before, total);
     __syncthreads();
     const int32_t R = cta_padded_scan(total, E, align, base, warp_tot);
     for (int e = threadIdx.x; e < E; e += kRouteThreads) {
@@ -309,16 +376,16 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
     }
     if (tile == 0 && threadIdx.x == 0) offsets[E] = R;
     __syncthreads();
-    tile_mark(bitmap, e_reg, iters, p0, p1, k, t0, E, err_flag);
+    tile_mark(bitmap, e_reg, n, divk, E, err_flag);
     __syncthreads();
-    tile_scatter(bitmap, base, e_reg, iters, p0, p1, k, t0, E, slot_of, token_of);
+    tile_scatter(bitmap, base, e_reg, n, divk, p0, t0, E, slot_of, token_of);
 }
 
 }  // namespace
 
 size_t route_map_workspace_bytes_impl(int T, int E) {
     const int tiles = num_tiles(T) > 0 ? num_tiles(T) : 1;
-    return static_cast<size_t>(tiles) * static_cast<size_t>(E) * sizeof(int32_t);
+    return static_cast<size_t>(row_stride(tiles)) * static_cast<size_t>(E) * sizeof(int32_t);
 }
 
 }  // namespace tk
@@ -357,25 +424,26 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* tile_counts = static_cast<int32_t*>(workspace);
     const int tiles = num_tiles(T);
+    const int stride = row_stride(tiles);
     const int count_grid = tiles > 0 ? tiles : 1;
     cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
-                                 tile_counts, token_of, rmax, err_flag);
+                                 tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
-    if (tiles > 0 && tiles <= kFusedMaxTiles) {
+    if (tiles > 0 && static_cast<int64_t>(stride) * E <= kFusedMaxEntries) {
         const size_t smem = static_cast<size_t>(E) * (kTileWords + 3) * sizeof(uint32_t);
         err = launch_pdl(route_scan_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s,
-                         topk_idx, T, E, k, align, static_cast<const int32_t*>(tile_counts), tiles,
-                         counts, offsets, slot_of, token_of, err_flag);
+                         topk_idx, T, E, k, align, static_cast<const int32_t*>(tile_counts),
+                         stride, counts, offsets, slot_of, token_of, err_flag);
         return check_launch(err, "route_scan_scatter_kernel");
     }
-    err = launch_pdl(route_scan_kernel, dim3(1), dim3(scan_threads(E)), 0, s, tile_counts, tiles, E,
-                     align, counts, offsets);
+    err = launch_pdl(route_scan_kernel, dim3(1), dim3(scan_threads(E)), 0, s, tile_counts, tiles,
+                     stride, E, align, counts, offsets);
     if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
     if (tiles > 0) {
         const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
         err = launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
-                         T, E, k, static_cast<const int32_t*>(tile_counts),
+                         T, E, k, static_cast<const int32_t*>(tile_counts), stride,
                          static_cast<const int32_t*>(offsets), slot_of, token_of, err_flag);
         if (err != cudaSuccess) return check_launch(err, "route_scatter_kernel");
     }
@@ -389,11 +457,12 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
 // every byte of device memory and passes a component only its input and output buffers, or a
 // latency-critical loop where a cudaMalloc (which can synchronise the device) is not allowed.
 // For them the tile-count matrix lives in a fixed array compiled into this library. Every GPU
-// that loads the library reserves it (1 MiB) until the process exits.
+// that loads the library reserves it (2 MiB) until the process exits.
 //
 // The array's name is only a host-side stand-in in host code; its device address is looked up
 // with cudaGetSymbolAddress once per device (with that device current) on the first call on
-// that device, and cached. The kernels write every entry they later read, so nothing in the
+// that device, and cached for the life of the process (a device reset after that first call is
+// not supported: the cached address would be stale). The kernels write every entry they later read, so nothing in the
 // array has to start at zero. All calls on one device share the array: calls that can overlap
 // on the GPU (other streams, other host threads) race on it and must be serialised by the
 // caller.
@@ -401,7 +470,7 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
 #include <mutex>
 
 namespace {
-constexpr size_t kStaticScratchInts = 256 * 1024;  // 1 MiB of int32 tile counts
+constexpr size_t kStaticScratchInts = 512 * 1024;  // 2 MiB of int32 tile counts
 static __device__ __align__(256) int32_t tk_route_static_scratch[kStaticScratchInts];
 
 constexpr int kMaxDevices = 64;
@@ -444,9 +513,10 @@ extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, 
     const size_t need = route_map_workspace_bytes_impl(T, E) / sizeof(int32_t);
     if (need > kStaticScratchInts)
         return fail_arg("tk_route_map_static: T=%d, E=%d need %zu scratch entries but the built-in "
-                        "buffer holds %zu (at most %zu tiles of 256 tokens times E); use "
-                        "tk_route_map with a caller workspace", T, E, need, kStaticScratchInts,
-                        kStaticScratchInts / static_cast<size_t>(E));
+                        "buffer holds %zu (E times the tiles of %d tokens rounded up to a multiple "
+                        "of 4, at most %zu tiles here); use tk_route_map with a caller workspace",
+                        T, E, need, kStaticScratchInts, kTileTokens,
+                        kStaticScratchInts / static_cast<size_t>(E) / 4 * 4);
     if (counts == nullptr || offsets == nullptr)
         return fail_arg("tk_route_map_static: counts and offsets must not be NULL");
     if (T > 0 && (topk_idx == nullptr || slot_of == nullptr))
@@ -457,18 +527,19 @@ extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, 
     if (st != TK_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int tiles = num_tiles(T);
+    const int stride = row_stride(tiles);
     const int count_grid = tiles > 0 ? tiles : 1;
     cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
-                                 tile_counts, token_of, rmax, err_flag);
+                                 tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
-    err = launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tile_counts, tiles, E,
-                     align, counts, offsets);
+    err = launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tile_counts, tiles,
+                     stride, E, align, counts, offsets);
     if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
     if (tiles > 0) {
         const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
         err = launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
-                         T, E, k, static_cast<const int32_t*>(tile_counts),
+                         T, E, k, static_cast<const int32_t*>(tile_counts), stride,
                          static_cast<const int32_t*>(offsets), slot_of, token_of, err_flag);
         if (err != cudaSuccess) return check_launch(err, "route_scatter_kernel");
     }
