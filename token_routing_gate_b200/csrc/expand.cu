@@ -27,8 +27,8 @@
 namespace tk {
 namespace {
 
-#ifndef TK_EXPAND_STORE_EVICT_FIRST
-#define TK_EXPAND_STORE_EVICT_FIRST 1
+#ifndef TK_EXPAND_STORE_POLICY   // L2 policy of the k stores: 0 none, 1 evict-normal, 2 evict-first, 3 evict-last
+#define TK_EXPAND_STORE_POLICY 2
 #endif
 
 constexpr uint32_t kCopyChunkBytes = 32768;  // bf16 bytes staged per bulk load
@@ -43,7 +43,7 @@ __device__ __forceinline__ void load_copy(void* dst, const void* src, uint32_t b
 }
 
 __device__ __forceinline__ void store_copy(void* dst, const void* src, uint32_t bytes, uint64_t policy) {
-    if (TK_EXPAND_STORE_EVICT_FIRST) bulk_store_hint(dst, src, bytes, policy);
+    if (TK_EXPAND_STORE_POLICY != 0) bulk_store_hint(dst, src, bytes, policy);
     else bulk_store(dst, src, bytes);
 }
 constexpr int kFp8Threads = 256;
@@ -71,7 +71,7 @@ expand_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ sl
     }
     const uint8_t* src = x + t * row_bytes;
     const uint32_t nchunks = (row_bytes + kCopyChunkBytes - 1) / kCopyChunkBytes;
-    const uint64_t policy = l2_policy_evict_first();
+    const uint64_t policy = l2_policy(TK_EXPAND_STORE_POLICY);
     for (uint32_t c = 0; c < nchunks; ++c) {
         const uint32_t off = c * kCopyChunkBytes;
         const uint32_t bytes = min(kCopyChunkBytes, row_bytes - off);
@@ -131,7 +131,7 @@ expand_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sl
     }
     const int nb_row = H / 128;
     const int nchunks = (H + chunk - 1) / chunk;
-    const uint64_t policy = l2_policy_evict_first();
+    const uint64_t policy = l2_policy(TK_EXPAND_STORE_POLICY);
     for (int c = 0; c < nchunks; ++c) {
         const int ch0 = c * chunk;
         const int chn = min(chunk, H - ch0);

@@ -148,9 +148,18 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     return p;
 }
 
-// Policy by number, for the kernels' tuning switches: 0 none, 1 evict-normal, 2 evict-first.
+// Evict-last policy: lines kept ahead of evict-normal and evict-first ones.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Policy by number, for the kernels' tuning switches: 0 none, 1 evict-normal, 2 evict-first,
+// 3 evict-last.
 __device__ __forceinline__ uint64_t l2_policy(int which) {
-    return which == 2 ? l2_policy_evict_first() : l2_policy_evict_normal();
+    return which == 2 ? l2_policy_evict_first()
+                      : (which == 3 ? l2_policy_evict_last() : l2_policy_evict_normal());
 }
 
 // bulk_load with an L2 cache-policy hint.
