@@ -744,6 +744,11 @@ def run_ep(args, wl):
     scale_b = 4 * (H // 128) if args.ep_dtype == "fp8" else 0
     disp_bytes = T * 2 * H + sent_rows * (row_out + scale_b + 8 * k) + T * k * 8
     comb_bytes = sent_rows * 2 * H + T * 2 * H
+    # destinations: every pair is a local choice on exactly one rank, so the experts' rows read
+    # are T*k rows; each received row's choices and weights are read and its partial written
+    # (the route maps' index traffic is small and not counted)
+    dest_bytes = T * k * 2 * H + sent_rows * (k * 8 + 2 * H)
+    peak, peak_kind = load_peak()
     line = {"metric": f"expert-parallel dispatch + combine tokens/s, {G} ranks on one GPU",
             "op": "ep", "value": T / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -758,8 +763,13 @@ def run_ep(args, wl):
                            / (kernel_us["dispatch"] * 1e3),
                            "combine": (sent0 * 2 * H + Tr * 2 * H) / (kernel_us["combine"] * 1e3)},
             "hbm_gbs": {"dispatch": disp_bytes / (phase_us["dispatch"] * 1e3),
+                        "experts": dest_bytes / (phase_us["experts"] * 1e3),
                         "combine": comb_bytes / (phase_us["combine"] * 1e3)},
-            "bytes": {"dispatch": disp_bytes, "combine": comb_bytes},
+            "experts_frac": {"value": dest_bytes / (phase_us["experts"] * 1e3) / peak, "peak": peak,
+                             "peak_kind": peak_kind,
+                             "note": "destination phase (route maps + tk_reduce_masked of every "
+                                     "rank's received rows) against the HBM peak"},
+            "bytes": {"dispatch": disp_bytes, "experts": dest_bytes, "combine": comb_bytes},
             "clocks": clocks.summary(), "gpu_launches": None, "system": system_info(dev)}
     print(json.dumps(line), flush=True)
     return 0

@@ -81,6 +81,33 @@ def test_global_balance_stats_over_rank_shards(shards):
     assert abs(loss.item() - lr) <= ULP32 * abs(lr)
 
 
+@pytest.mark.parametrize("k", [8, 12, 16, 24, 32])
+def test_reduce_mixed_valid_counts(k):
+    """Tokens keep a random number of their k choices (the rest masked -1), so consecutive units
+    of the reduce's row ring need very different amounts of it -- a unit of more than half the
+    ring right after a small one included. Both forms match the oracle, no wait gives up."""
+    rng = np.random.default_rng(k)
+    T, E, H = 1500, 64, 2304
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    keep = rng.integers(0, k + 1, T)
+    keep[rng.random(T) < 0.3] = k                     # many fully valid tokens among them
+    for t in range(T):
+        idx[t, rng.permutation(k)[keep[t]:]] = -1
+    w = rng.random((T, k)).astype(np.float32)
+    counts, offsets, slot_of, token_of, rc = oracle.route_map(idx, E, 1)
+    rows = max(int(offsets[-1]), 1)
+    y = torch.randn(rows, H, generator=torch.Generator().manual_seed(k)).to(torch.bfloat16)
+    ref = oracle.reduce(bf16_bits(y), slot_of, w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    yd, sd, wd = y.cuda(), torch.from_numpy(slot_of).cuda(), torch.from_numpy(w).cuda()
+    a = tk.reduce(yd, sd, wd, err_flag=err)
+    b = tk.reduce(yd, sd, wd, err_flag=err, masked=True)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    np.testing.assert_array_equal(bf16_bits(a), ref)
+    np.testing.assert_array_equal(bf16_bits(b), ref)
+
+
 @pytest.mark.parametrize("case", ["dense", "tp8", "ep_like", "ragged"])
 def test_reduce_masked_equals_reduce(case):
     wl = {"dense": W.V3.with_(T=3000, H=1024), "tp8": W.V3.with_(T=4000, H=512),

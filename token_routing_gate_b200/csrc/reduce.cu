@@ -47,12 +47,25 @@ namespace {
 #define TK_REDUCE_STAGE_KB 32
 #endif
 
+#ifndef TK_REDUCE_MASKED_VECS_PER_THREAD
+#define TK_REDUCE_MASKED_VECS_PER_THREAD 2
+#endif
+
 constexpr int kConsumerWarps = TK_REDUCE_CONSUMER_WARPS;
-constexpr int kVecs = TK_REDUCE_VECS_PER_THREAD;        // 8-channel vectors per consumer thread
+// 8-channel vectors per consumer thread and unit: the dense reduce (every pair valid) and the
+// masked form (tk_reduce_masked: most pairs -1, so a unit's few valid rows are small and wider
+// units carry the per-unit work over more bytes)
+constexpr int kVecsDense = TK_REDUCE_VECS_PER_THREAD;
+constexpr int kVecsMasked = TK_REDUCE_MASKED_VECS_PER_THREAD;
 constexpr int kRedThreads = 32 * (1 + kConsumerWarps);
-constexpr int kChunkCh = 8 * 32 * kConsumerWarps * kVecs;  // channels per unit
-constexpr int kChunkBytes = kChunkCh * 2;                  // bf16 bytes of one row chunk
 constexpr int kStageBudget = TK_REDUCE_STAGE_KB * 1024;    // shared bytes of row data per CTA
+
+// Channels of one unit and bf16 bytes of one of its row chunks, for kV vectors per thread.
+template <int kV>
+struct UnitShape {
+    static constexpr int ch = 8 * 32 * kConsumerWarps * kV;
+    static constexpr int bytes = ch * 2;
+};
 constexpr int kRingEntries = 16;                           // units in flight at most
 
 // One unit's entry in the ring: its valid rows sit back to back at `off`, in slot order, and
@@ -73,7 +86,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Bytes of the row ring: the budget, and at least one unit with all k rows valid.
-int ring_bytes_for(int k) { return k * kChunkBytes > kStageBudget ? k * kChunkBytes : kStageBudget; }
+int ring_bytes_for(int k, int chunk_bytes) {
+    return k * chunk_bytes > kStageBudget ? k * chunk_bytes : kStageBudget;
+}
 
 size_t smem_bytes(int ring) {
     return static_cast<size_t>(ring) + kRingEntries * sizeof(EntryMeta) +
@@ -140,10 +155,12 @@ struct RankRows {
 
 // kStep: step each unit's (token, chunk) and ring offset by O(1) updates instead of 64-bit
 // division and modulo (the tk_reduce_masked form; see the entry points).
-template <class Rows, bool kStep>
+template <class Rows, bool kStep, int kVecs>
 __global__ void __launch_bounds__(kRedThreads)
 reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, int T, int k, int H,
               int ring, uint8_t* __restrict__ out, int32_t* err_flag) {
+    constexpr int kChunkCh = UnitShape<kVecs>::ch;
+    constexpr int kChunkBytes = UnitShape<kVecs>::bytes;
     extern __shared__ __align__(128) uint8_t sm[];
     uint8_t* data = sm;                                                    // [ring] row bytes
     EntryMeta* meta = reinterpret_cast<EntryMeta*>(sm + ring);             // [kRingEntries]
@@ -240,7 +257,11 @@ reduce_kernel(const __grid_constant__ Rows rows, const float* __restrict__ w, in
             }
             const uint64_t h_end = h + need;
             int ok = 1;
-            while (it - rel >= kRingEntries || h_end - tail > static_cast<uint64_t>(ring)) {
+            // Space: the bytes from the oldest unreleased unit to this unit's end must fit in the
+            // ring. Once every earlier unit is released nothing is live, and the unit fits even
+            // when the gap skipped by wrapping makes that span longer than the ring (a unit of
+            // more than half the ring after a smaller one would otherwise wait forever).
+            while (it - rel >= kRingEntries || (rel < it && h_end - tail > static_cast<uint64_t>(ring))) {
                 const int e = rel % kRingEntries;
                 if (lane == 0) ok = mbar_wait_bounded(&empty[e], static_cast<uint32_t>(rel / kRingEntries) & 1u) ? 1 : 0;
                 ok = __shfl_sync(kFullMask, ok, 0);
@@ -341,7 +362,7 @@ struct LaunchShape {
 
 // Launch shape for k on the current device, worked out once per row source (the kernel's
 // shared-memory limit is raised to the largest size any k needs).
-template <class Rows, bool kStep>
+template <class Rows, bool kStep, int kVecs>
 cudaError_t launch_shape(int k, LaunchShape& out) {
     static LaunchShape shapes[kMaxDevices][TK_MAX_TOPK + 1];
     static std::atomic<bool> ready[kMaxDevices][TK_MAX_TOPK + 1];
@@ -353,17 +374,17 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
     }
     std::lock_guard<std::mutex> lock(setup_mutex());
     if (!ready[dev][k].load(std::memory_order_relaxed)) {
-        const int ring = ring_bytes_for(k);
+        const int ring = ring_bytes_for(k, UnitShape<kVecs>::bytes);
         const size_t smem = smem_bytes(ring);
         cudaError_t err = cudaSuccess;
         if (static_cast<int>(smem) > configured_smem[dev]) {
-            err = cudaFuncSetAttribute(reduce_kernel<Rows, kStep>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(reduce_kernel<Rows, kStep, kVecs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
             if (err != cudaSuccess) return err;
             configured_smem[dev] = static_cast<int>(smem);
         }
         int per_sm = 0;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows, kStep>, kRedThreads, smem);
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows, kStep, kVecs>, kRedThreads, smem);
         if (err != cudaSuccess) return err;
         shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
         shapes[dev][k].ring = ring;
@@ -373,18 +394,19 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
     return cudaSuccess;
 }
 
-template <class Rows, bool kStep = false>
+template <class Rows, bool kStep = false, int kVecs = kVecsDense>
 cudaError_t launch_reduce(const Rows& rows, const float* w, int T, int k, int H, void* out,
                           int32_t* err_flag, void* stream, const char** what) {
     *what = "reduce_kernel setup";
     LaunchShape shape;
-    const cudaError_t e = launch_shape<Rows, kStep>(k, shape);
+    const cudaError_t e = launch_shape<Rows, kStep, kVecs>(k, shape);
     if (e != cudaSuccess) return e;
     *what = "reduce_kernel";
+    constexpr int kChunkCh = UnitShape<kVecs>::ch;
     const int64_t chunks = (H + kChunkCh - 1) / kChunkCh;
     const int64_t units = static_cast<int64_t>(T) * chunks;
     const int grid = static_cast<int>(units < shape.grid_cap ? units : shape.grid_cap);
-    return launch_pdl(reduce_kernel<Rows, kStep>, dim3(grid), dim3(kRedThreads), smem_bytes(shape.ring),
+    return launch_pdl(reduce_kernel<Rows, kStep, kVecs>, dim3(grid), dim3(kRedThreads), smem_bytes(shape.ring),
                       static_cast<cudaStream_t>(stream), rows, w, T, k, H, shape.ring,
                       static_cast<uint8_t*>(out), err_flag);
 }
@@ -410,7 +432,8 @@ tk_status reduce_entry(const char* name, const void* y, int64_t y_rows, const in
         return fail_arg("%s: y and out must be 16-byte aligned", name);
     const SlotRows rows{static_cast<const uint8_t*>(y), y_rows, slot_of};
     const char* what = "";
-    const cudaError_t err = launch_reduce<SlotRows, kStep>(rows, w, T, k, H, out, err_flag, stream, &what);
+    const cudaError_t err = launch_reduce<SlotRows, kStep, kStep ? kVecsMasked : kVecsDense>(
+        rows, w, T, k, H, out, err_flag, stream, &what);
     return check_launch(err, what);
 }
 
