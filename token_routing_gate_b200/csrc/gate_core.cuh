@@ -40,55 +40,6 @@ __device__ __forceinline__ float key_sigmoidf(float l) {
     return __fdiv_rn(1.0f, __fadd_rn(1.0f, key_expf(-l)));
 }
 
-// ---- fp64 arithmetic of the sigmoid weights. A weight only has to come within a few fp64 ulps
-// of s_j / sum(s) before it is rounded to fp32 (it then rounds like the oracle's fp64 value
-// except with probability ~2^-27), so these need not be correctly rounded.
-
-// e^x in fp64: Cody-Waite reduction by ln 2 (ln 2 split into a 21-bit high part, so n * hi is
-// exact for |n| < 2^11, and the fp64 remainder), degree-13 Taylor polynomial of e^r on
-// |r| <= ln2/2 (truncation below 6e-18) with coefficients 1/i! rounded to fp64, Horner with
-// fma, then 2^n in two exact steps. e^x overflows to +inf above ln(DBL_MAX) and is 0 below
-// -746, as a correctly rounded exponential does; NaN passes through.
-__device__ __forceinline__ double weight_exp(double x) {
-    if (x != x) return x;
-    if (x > 709.782712893384) return INFINITY;
-    if (x < -746.0) return 0.0;
-    const double n = rint(x * 0x1.71547652b82fep+0);
-    double r = fma(-n, 0x1.62e42p-1, x);
-    r = fma(-n, 0x1.fdf473de6af28p-22, r);
-    double p = 0x1.6124613a86d09p-33;     // 1/13!
-    p = fma(p, r, 0x1.1eed8eff8d898p-29);  // 1/12!
-    p = fma(p, r, 0x1.ae64567f544e4p-26);  // 1/11!
-    p = fma(p, r, 0x1.27e4fb7789f5cp-22);  // 1/10!
-    p = fma(p, r, 0x1.71de3a556c734p-19);  // 1/9!
-    p = fma(p, r, 0x1.a01a01a01a01ap-16);  // 1/8!
-    p = fma(p, r, 0x1.a01a01a01a01ap-13);  // 1/7!
-    p = fma(p, r, 0x1.6c16c16c16c17p-10);  // 1/6!
-    p = fma(p, r, 0x1.1111111111111p-7);   // 1/5!
-    p = fma(p, r, 0x1.5555555555555p-5);   // 1/4!
-    p = fma(p, r, 0x1.5555555555555p-3);   // 1/3!
-    p = fma(p, r, 0.5);
-    p = fma(p, r, 1.0);
-    p = fma(p, r, 1.0);
-    const int ni = static_cast<int>(n);    // [-1077, 1024]
-    const int n1 = ni / 2;
-    const int n2 = ni - n1;
-    return p * __hiloint2double((n1 + 1023) << 20, 0) * __hiloint2double((n2 + 1023) << 20, 0);
-}
-
-// 1/x in fp64 for x >= 2^-1000: the hardware's approximate reciprocal refined by two Newton
-// steps y += y (1 - x y) (each squares the relative error); IEEE division for huge or
-// infinite x.
-__device__ __forceinline__ double weight_rcp(double x) {
-    if (!(x < 0x1p+1000)) return 1.0 / x;
-    double y;
-    asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(x));
-    double e = fma(-x, y, 1.0);
-    y = fma(y, e, y);
-    e = fma(-x, y, 1.0);
-    return fma(y, e, y);
-}
-
 // Order-preserving map of an fp32 key to uint32 (larger key -> larger integer). -0 is folded
 // onto +0 and NaN onto -inf first, so float equality and integer equality agree.
 __device__ __forceinline__ uint32_t ordered_key(float key) {

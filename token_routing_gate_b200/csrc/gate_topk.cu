@@ -172,19 +172,17 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
             gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, idx_out, w_out);
             continue;
         }
-        // weights in fp64 (within a few fp64 ulps of the exact value), rounded once to fp32, so
-        // they round like the oracle's and the reduce that uses them agrees with it too
-        const double sd = chosen ? gate::weight_rcp(1.0 + gate::weight_exp(-static_cast<double>(l))) : 0.0;
+        // weights in fp64, rounded once to fp32, so they round like the oracle's and the reduce
+        // that uses them agrees with it too
+        const double sd = chosen ? 1.0 / (1.0 + exp(-static_cast<double>(l))) : 0.0;
         double denom = sd;
         if (renormalize) {
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) denom += __shfl_xor_sync(kFullMask, denom, off);
         }
         if (chosen) {
-            float w = static_cast<float>(sd);
-            if (renormalize)
-                w = denom == 0.0 ? 0.0f
-                    : static_cast<float>(denom >= 0x1p-1000 ? sd * gate::weight_rcp(denom) : sd / denom);
+            const float w = !renormalize ? static_cast<float>(sd)
+                                         : (denom == 0.0 ? 0.0f : static_cast<float>(sd / denom));
             idx_out[rank] = e;
             w_out[rank] = w;
         }
