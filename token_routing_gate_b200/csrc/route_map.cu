@@ -330,10 +330,10 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     int e_reg[kPairsPerThread];
     load_tile(topk_idx, p0, n, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
-    for (int e = threadIdx.x; e < E; e += kRouteThreads)
-        base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(e) * stride + tile];
     __syncthreads();
     tile_mark(bitmap, e_reg, n, divk, E, err_flag);
+    for (int e = threadIdx.x; e < E; e += kRouteThreads)
+        base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(e) * stride + tile];
     __syncthreads();
     tile_scatter(bitmap, base, e_reg, n, divk, p0, t0, E, slot_of, token_of);
 }
@@ -363,6 +363,9 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
     int e_reg[kPairsPerThread];
     load_tile(topk_idx, p0, n, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
+    __syncthreads();
+    // the tile's bitmap does not depend on the scan: mark it while the row sums' loads are out
+    tile_mark(bitmap, e_reg, n, divk, E, err_flag);
     // per expert: the count over the tiles before this one, and the row total
     row_sums(tile_counts, stride, E, tile, before, total);
     __syncthreads();
@@ -375,8 +378,6 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
         base[e] += before[e];
     }
     if (tile == 0 && threadIdx.x == 0) offsets[E] = R;
-    __syncthreads();
-    tile_mark(bitmap, e_reg, n, divk, E, err_flag);
     __syncthreads();
     tile_scatter(bitmap, base, e_reg, n, divk, p0, t0, E, slot_of, token_of);
 }
