@@ -44,11 +44,12 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for cpu_baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--op", choices=["step", "backward", "stats", "ep"], default="step",
+    p.add_argument("--op", choices=["step", "backward", "stats", "ep", "boundary"], default="step",
                    help="step: the forward path (the benchmark's headline); backward: reduce and "
                         "expand backward; stats: load-balance statistics and the TP mask; ep: "
                         "expert-parallel dispatch/combine of the batch over --ep-ranks ranks run "
-                        "on one GPU")
+                        "on one GPU; boundary: reduce and expand each timed right after different "
+                        "predecessors (itself, the other, a write that leaves L2 dirty, a read)")
     p.add_argument("--ep-ranks", type=int, default=8, help="ranks of the --op ep run")
     p.add_argument("--ep-tokens", type=int, default=None,
                    help="tokens per rank of the --op ep run (default: the workload's T, i.e. every "
@@ -775,6 +776,70 @@ def run_ep(args, wl):
     return 0
 
 
+def run_boundary(args, wl):
+    """tk_reduce and tk_expand of the workload, each launch timed on its own (events around it)
+    right after a predecessor: the same call, the other call, a 256 MB or 64 MB write that leaves
+    L2 full of dirty lines, a 256 MB read that leaves it clean. Median of K launches each. Shows
+    what the step's order costs: the reduce follows expand, whose last writes are still dirty in
+    L2 and are written back while the reduce reads."""
+    import torch
+    from token_routing_gate_b200 import tk
+    from token_routing_gate_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = torch.cuda.current_stream(dev)
+    logits, bias = W.gate_inputs(wl, dev)
+    x = W.activations(wl, dev)
+    R = tk.max_rows(wl.T, wl.E, wl.k, wl.align)
+    y = W.expert_outputs(wl, dev, rows=R)
+    idx, w = tk.gate_topk(logits, wl.k, wl.score, bias)
+    rm = tk.route_map(idx, wl.E, wl.align)
+    xe = torch.empty(R, wl.H, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+    big = torch.empty(256 << 18, dtype=torch.float32, device=dev)   # 256 MB
+    src = torch.ones_like(big)
+
+    def reduce():
+        tk.reduce(y, rm.slot_of, w, out=out, stream=s)
+
+    def expand():
+        tk.expand(x, rm, wl.E, wl.k, "bf16", out=xe, stream=s)
+
+    preds = {"itself": None, "reduce": reduce, "expand": expand,
+             "dirty_write_256MB": lambda: big.fill_(1.0),
+             "dirty_write_64MB": lambda: big[: 64 << 18].fill_(1.0),
+             "clean_read_256MB": lambda: torch.sum(src)}
+    K = max(args.steps, 5)
+    res = {}
+    with ClockSampler(dev.index) as clocks:
+        for name, op in (("reduce", reduce), ("expand", expand)):
+            res[name] = {}
+            for pname, prep in preds.items():
+                prep = prep or op
+                ts = []
+                for i in range(K + args.warmup):
+                    prep()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(s)
+                    op()
+                    b.record(s)
+                    torch.cuda.synchronize(dev)
+                    if i >= args.warmup:
+                        ts.append(a.elapsed_time(b) * 1e3)
+                res[name][pname] = statistics.median(ts)
+    ab = algorithmic_bytes(wl, int(rm.offsets[-1].item()))
+    line = {"metric": "reduce / expand us after different predecessors", "op": "boundary",
+            "value": res["reduce"]["expand"], "unit": "us", "n_gpus": 1, "steps": K,
+            "warmup": args.warmup, "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "E": wl.E, "k": wl.k, "H": wl.H},
+            "median_us": res,
+            "bytes": {"reduce": ab["reduce"], "expand": ab["expand"]},
+            "clocks": clocks.summary(), "gpu_launches": None, "system": system_info(dev)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     from token_routing_gate_b200 import workloads as W
@@ -785,6 +850,8 @@ def main():
         return run_reference(args, wl)
     if args.op == "ep":
         return run_ep(args, wl)
+    if args.op == "boundary":
+        return run_boundary(args, wl)
     if args.op != "step":
         return run_op(args, wl)
     return run_tk(args, wl)

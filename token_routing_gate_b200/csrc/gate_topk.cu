@@ -41,9 +41,10 @@ constexpr int kGateWarps = 8;  // tokens per CTA
 // fewer than k lanes holding an expert send the token down the full path: every exact key, a
 // per-lane sort and k rounds over the sorted lists.
 //
-// Weights are computed in fp64 and rounded once to fp32, as in the oracle: fp32 weights
-// within the 1e-6 bar but a few ulps off the oracle's would move reduce outputs that nearly
-// cancel by more than one bf16 ulp.
+// Weights are computed in fp64 and rounded once to fp32, so they are the correctly rounded
+// fp32 values of the defining quotient except in rare halfway cases: fp32 weights within 1e-6
+// relative but a few ulps off those values would move reduce outputs that nearly cancel by more
+// than one bf16 ulp.
 __device__ __forceinline__ float filter_margin(const float* b, int epl, bool has_bias, bool* ok) {
     if (!has_bias) {
         *ok = true;
@@ -172,8 +173,8 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
             gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, idx_out, w_out);
             continue;
         }
-        // weights in fp64, rounded once to fp32, so they round like the oracle's and the reduce
-        // that uses them agrees with it too
+        // weights in fp64, rounded once to fp32 (the correctly rounded values of s_j / sum s,
+        // except in rare halfway cases), so the reduce that uses them is reproducible too
         const double sd = chosen ? 1.0 / (1.0 + exp(-static_cast<double>(l))) : 0.0;
         double denom = sd;
         if (renormalize) {
