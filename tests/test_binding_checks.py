@@ -115,5 +115,11 @@ def test_ep_buffers_are_checked(tk):
     with pytest.raises(TypeError, match="idx"):
         tk.ep_peer(cuda_like(10, 64, dtype=torch.bfloat16), cuda_like(10, 2, dtype=torch.int64),
                    cuda_like(10, 2), 0, 10)
+    # a descriptor of buffers already checked takes their addresses as they are
+    x, idx, w = (torch.zeros(10, 64, dtype=torch.bfloat16), torch.zeros(10, 2, dtype=torch.int32),
+                 torch.zeros(10, 2))
+    again = tk.ep_peer(x, idx, w, 7, 10, checked=True)
+    assert (again.x, again.idx, again.w, again.scale, again.base_row) == (
+        x.data_ptr(), idx.data_ptr(), w.data_ptr(), None, 7)
     peer = tk.ep_peer(123456, 234560, 345600, 5, 10)   # raw addresses pass unchecked
     assert peer.x == 123456 and peer.idx == 234560 and peer.rows == 10 and peer.base_row == 5

@@ -31,7 +31,7 @@ def vr_env(monkeypatch):
         out.send_counts.copy_(torch.tensor(counts, dtype=torch.int32))
         return out
 
-    def fake_peer(x, idx, w, base_row, rows, scale=None):
+    def fake_peer(x, idx, w, base_row, rows, scale=None, checked=False):
         return {"x": x, "base_row": int(base_row), "rows": int(rows)}
 
     def fake_dispatch(x, idx, w, layout, E, peers, out_dtype="bf16", err_flag=None, stream=None):

@@ -118,6 +118,14 @@ ep_dispatch_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict
     }
     __syncwarp();
     pdl_wait();
+    const uint8_t* src = x + t * row_bytes;
+    // the first piece of the row does not depend on where it goes: start its load before the
+    // destinations are worked out
+    if (lane == 0) {
+        const uint32_t bytes0 = min(kEpChunkBytes, row_bytes);
+        mbar_arrive_expect_tx(&bar, bytes0);
+        bulk_load(stage, src, bytes0, &bar);
+    }
     const int64_t my_row = dest_row(dest_slot, send_offsets, peers, t, G, lane, err_flag);
     int e = -1;
     float wt = 0.0f;
@@ -127,9 +135,7 @@ ep_dispatch_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict
         if (e < -1 || e >= E) e = -1;   // tk_ep_layout flags these
     }
     write_choices(peers, my_row, G, k, E / G, e, wt, lane);
-    if (__ballot_sync(kFullMask, my_row >= 0) == 0u) return;
 
-    const uint8_t* src = x + t * row_bytes;
     const uint32_t nchunks = (row_bytes + kEpChunkBytes - 1) / kEpChunkBytes;
     for (uint32_t c = 0; c < nchunks; ++c) {
         const uint32_t off = c * kEpChunkBytes;
@@ -139,9 +145,9 @@ ep_dispatch_bf16_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict
             if (c > 0) {
                 bulk_wait_read_all();      // previous piece fully read by its stores
                 fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&bar, bytes);
+                bulk_load(stage, src + off, bytes, &bar);
             }
-            mbar_arrive_expect_tx(&bar, bytes);
-            bulk_load(stage, src + off, bytes, &bar);
             ok = mbar_wait_bounded(&bar, c & 1u) ? 1 : 0;
             if (!ok) {
                 flag_error(err_flag, TK_DEVERR_TIMEOUT);
@@ -182,6 +188,13 @@ ep_dispatch_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict
     }
     __syncthreads();
     pdl_wait();
+    // the first piece of the row does not depend on where it goes: start its load before the
+    // destinations are worked out
+    if (tid == 0) {
+        const uint32_t bytes0 = static_cast<uint32_t>(min(chunk, H)) * 2u;
+        mbar_arrive_expect_tx(&bar, bytes0);
+        bulk_load(xin, x + t * H, bytes0, &bar);
+    }
     if (warp == 0) {
         const int64_t my_row = dest_row(dest_slot, send_offsets, peers, t, G, lane, err_flag);
         if (lane < G) rows[lane] = my_row;
@@ -195,9 +208,6 @@ ep_dispatch_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict
         write_choices(peers, my_row, G, k, E / G, e, wt, lane);
     }
     __syncthreads();
-    bool any = false;
-    for (int d = 0; d < G; ++d) any |= rows[d] >= 0;
-    if (!any) return;
 
     const int nb_row = H / 128;
     const int nchunks = (H + chunk - 1) / chunk;
@@ -205,10 +215,12 @@ ep_dispatch_fp8_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict
         const int ch0 = c * chunk;
         const int chn = min(chunk, H - ch0);
         if (tid == 0) {
-            if (c > 0) bulk_wait_read_all();
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(chn) * 2u);
-            bulk_load(xin, x + t * H + ch0, static_cast<uint32_t>(chn) * 2u, &bar);
+            if (c > 0) {
+                bulk_wait_read_all();
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(chn) * 2u);
+                bulk_load(xin, x + t * H + ch0, static_cast<uint32_t>(chn) * 2u, &bar);
+            }
             int ok = mbar_wait_bounded(&bar, static_cast<uint32_t>(c) & 1u) ? 1 : 0;
             if (!ok) {
                 flag_error(err_flag, TK_DEVERR_TIMEOUT);

@@ -67,9 +67,15 @@ class RankBuffers:
         self.idx = alloc((rows, k), torch.int32)
         self.w = alloc((rows, k), torch.float32)
         self.partial = alloc((rows, H), torch.bfloat16)
+        self._checked = False
 
     def peer(self, base_row):
-        return tk.ep_peer(self.x, self.idx, self.w, base_row, self.rows, scale=self.scale)
+        """Descriptor of these buffers for a source writing from base_row on. The buffers are
+        checked on the first call only (a step builds G descriptors per source, and
+        re-checking every tensor each time cost more host time than a dispatch kernel takes)."""
+        checked, self._checked = self._checked, True
+        return tk.ep_peer(self.x, self.idx, self.w, base_row, self.rows, scale=self.scale,
+                          checked=checked)
 
 
 def local_combine(bufs, n, E_local, align, expert_fn, d, stream=None):

@@ -403,9 +403,16 @@ def ep_layout(topk_idx, E, G, out=None, err_flag=None, stream=None):
     return out
 
 
-def ep_peer(x, idx, w, base_row, rows, scale=None):
-    """Descriptor of one destination's receive buffers: tensors or raw device addresses."""
+def _raw(t):
+    return None if t is None else (t if isinstance(t, int) else t.data_ptr())
+
+
+def ep_peer(x, idx, w, base_row, rows, scale=None, checked=False):
+    """Descriptor of one destination's receive buffers: tensors or raw device addresses.
+    checked=True: the same tensors passed an earlier call's checks, only their addresses are read."""
     rows = int(rows)
+    if checked:
+        return EpPeer(_raw(x), _raw(scale), _raw(idx), _raw(w), int(base_row), rows)
     return EpPeer(_addr(x, (BF16,) + E4M3, rows, "x"), _addr(scale, F32, rows, "scale"),
                   _addr(idx, I32, rows, "idx"), _addr(w, F32, rows, "w"), int(base_row), rows)
 
