@@ -137,3 +137,40 @@ def test_approximate_sigmoid_within_the_filter_bound():
     worst = float(err.item())
     print(f"largest |approximate - exact| logistic value: {worst:.3e} ({np.log2(worst):.2f} in log2)")
     assert worst < 2.0 ** -17
+
+
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+def test_candidate_keys_spanning_many_binades(score):
+    """Candidate keys that lie many binades apart (their integer images further apart than the
+    one-reduction rounds can pack), so the selection takes the two-reduction rounds; half the
+    tokens stay in one binade as a control."""
+    rng = np.random.default_rng(21 + (score == "sigmoid"))
+    T, E, k = 3000, 256, 8
+    logits = (rng.standard_normal((T, E)) - 6.0).astype(np.float32)
+    bias = None
+    if score == "softmax":
+        for t in range(0, T, 2):  # top 12 logits 4^j: 1 ... 4^11, spread over 22 binades
+            logits[t, rng.choice(E, 12, replace=False)] = 4.0 ** np.arange(12)
+    else:
+        bias = np.zeros(E, np.float32)
+        top = rng.choice(E, 12, replace=False)
+        bias[top] = 10.0 ** np.linspace(-2.0, 5.0, 12)  # keys from about 0.01 to 1e5
+        logits[1::2, top] = 4.0                          # the control tokens: sigmoid ~ 1 everywhere
+    _check(logits, bias, k, score)
+
+
+@pytest.mark.parametrize("renormalize", [True, False])
+@pytest.mark.parametrize("k", [8, 6, 5, 3])
+def test_weight_batches_with_full_path_tokens(k, renormalize):
+    """Enough tokens that each warp routes several and computes their weights together (32/k
+    tokens per pass), with every third token sent down the full path (40 equal top keys) in the
+    middle of a batch."""
+    rng = np.random.default_rng(40 + k + renormalize)
+    T, E = 20000, 256
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    tied = rng.choice(E, 40, replace=False)
+    bias[tied] = 0.05
+    logits[::3, :] -= 4.0
+    logits[::3][:, tied] = 3.0
+    _check(logits, bias, k, "sigmoid", renormalize)

@@ -130,10 +130,12 @@ __device__ __forceinline__ void approx_images(const float (&lg)[EPL], const floa
 // of two >= k, the minimum over G groups of 32/G adjacent lanes of each group's maximum (each
 // group contributes one value >= it). 0 when some group holds no expert.
 __device__ __forceinline__ uint32_t group_threshold(uint32_t v, int k) {
-    int width = 32;  // lanes per group
-    while (width > 1 && 32 / width < k) width >>= 1;
-    for (int off = 1; off < width; off <<= 1) v = max(v, __shfl_xor_sync(kFullMask, v, off));
-    for (int off = width; off < 32; off <<= 1) v = min(v, __shfl_xor_sync(kFullMask, v, off));
+    const int width = 32 >> (32 - __clz(k - 1));  // lanes per group: 32 / G (k in [1, 32])
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_xor_sync(kFullMask, v, off);
+        v = off < width ? max(v, o) : min(v, o);
+    }
     return v;
 }
 
@@ -158,10 +160,12 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 }
 
 // One warp's shared scratch: the candidates (expert, logit bits) in (slot of the lane's list,
-// lane) order, and the chosen experts by rank.
+// lane) order, and the chosen experts with their logits by (token of the batch, rank): token q's
+// rank-j choice at entry q*k + j.
 struct Candidates {
     uint2 el[32];
     int by_rank[32];
+    float l_by_rank[32];
 };
 
 // Ballots of the lane's experts whose image is >= cut; returns their number (warp-uniform).
@@ -231,6 +235,36 @@ __device__ __forceinline__ int select_topk(uint64_t (&v)[EPL], int k, int lane) 
         }
     }
     return my_e;
+}
+
+// Outputs of a batch of n consecutive tokens (n*k <= 32) with logistic scores, whose choices sit
+// in c.by_rank / c.l_by_rank: lane q*k + j takes token q's rank-j choice, computes its unbiased
+// score 1 / (1 + e^-l) in double, adds the k scores of its token in rank order when renormalising
+// (the order of the defining sum), and writes entry q*k + j of the batch's outputs (consecutive
+// in idx_out and w_out), rounded once to fp32. One pass serves up to 32/k tokens, so the double
+// arithmetic runs on up to every lane instead of k of them per token.
+__device__ __forceinline__ void write_batch(const Candidates& c, int n, int k, int renormalize, int lane,
+                                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+    __syncwarp();  // the batch's choices are in c
+    const bool mine = lane < n * k;
+    double s = 0.0;
+    int e = 0;
+    if (mine) {
+        e = c.by_rank[lane];
+        s = 1.0 / (1.0 + exp(-static_cast<double>(c.l_by_rank[lane])));
+    }
+    double denom = 1.0;
+    if (renormalize) {
+        const int first = lane - lane % k;  // this token's rank-0 lane (mod 32 past the batch)
+        denom = 0.0;
+        for (int j = 0; j < k; ++j) denom += __shfl_sync(kFullMask, s, first + j);
+    }
+    if (mine) {
+        idx_out[lane] = e;
+        w_out[lane] = !renormalize ? static_cast<float>(s)
+                                   : (denom == 0.0 ? 0.0f : static_cast<float>(s / denom));
+    }
+    __syncwarp();  // c may be refilled
 }
 
 // Weights of the chosen experts (double, rounded once to fp32); lanes j < k write idx_out[j]

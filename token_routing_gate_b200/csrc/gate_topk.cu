@@ -81,14 +81,17 @@ __device__ __forceinline__ void prefetch_row(const float* row, int E, int lane, 
 // One warp per token. The grid is one wave of resident warps and the T tokens are split evenly
 // over the nwarps warps (warp w takes tokens [w*T/nwarps, (w+1)*T/nwarps), so warps differ by
 // at most one token and every SM gets the same work); the next token's logits are loaded while
-// the current one is processed. EPL = experts held per lane (E <= 32 * EPL).
-template <int EPL>
+// the current one is processed. EPL = experts held per lane (E <= 32 * EPL); kFull: E is exactly
+// 32 * EPL, so no lane's expert is absent and E is a constant. With logistic scores a warp keeps
+// the choices of up to 32/k consecutive tokens and computes their weights in one pass.
+template <int EPL, bool kFull>
 __global__ void __launch_bounds__(kGateWarps * 32, EPL <= 8 ? 4 : 1)
-gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
+gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E_in,
                  int k, int score_fn, int renormalize, int nwarps,
                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     __shared__ gate::Candidates cands[kGateWarps];
     pdl_wait();
+    const int E = kFull ? 32 * EPL : E_in;
     const int lane = threadIdx.x & 31;
     const int64_t wid = static_cast<int64_t>(blockIdx.x) * kGateWarps + (threadIdx.x >> 5);
     if (wid >= nwarps) return;
@@ -98,6 +101,7 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
     gate::Candidates& cand = cands[threadIdx.x >> 5];
     const bool has_bias = bias != nullptr;
     const bool sigmoid = score_fn == TK_SCORE_SIGMOID;
+    const int batch = sigmoid ? 32 / k : 1;  // tokens per weight pass
 
     float b[EPL];  // this lane's selection biases, shared by all tokens
 #pragma unroll
@@ -108,16 +112,12 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
     bool can_filter;
     const float eps = filter_margin(b, EPL, has_bias, &can_filter);
     float lg[EPL];  // logits of the token being routed, then of the next one (prefetch)
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = i * 32 + lane;
-        lg[i] = e < E ? logits[t_begin * E + e] : 0.0f;
-    }
+    prefetch_row<EPL>(logits + t_begin * E, E, lane, lg);
 
+    int64_t t_batch = t_begin;  // first token of the open weight batch
     for (int64_t t = t_begin; t < t_end; ++t) {
         const float* row = logits + t * E;
-        int32_t* idx_out = topk_idx + t * k;
-        float* w_out = topk_w + t * k;
+        const int slot = static_cast<int>(t - t_batch);
         int C = 33;  // > 32: full path
         if (can_filter) {
             uint32_t u[EPL], bal[EPL];
@@ -138,59 +138,78 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
             gate::build_keys<EPL>(lg, b, has_bias, E, lane, v);
             if (t + 1 < t_end) prefetch_row<EPL>(row + E, E, lane, lg);
             const int my_e = gate::select_topk<EPL>(v, k, lane);
-            gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, idx_out, w_out);
-            continue;
-        }
-        // the candidates are captured: start the next token's loads
-        if (t + 1 < t_end) prefetch_row<EPL>(row + E, E, lane, lg);
-        // exact keys of the candidates, one per lane
-        int e = 0;
-        float l = 0.0f;
-        uint32_t hi = 0, lo = 0;
-        if (lane < C) {
-            const uint2 el = cand.el[lane];
-            e = static_cast<int>(el.x);
-            l = __uint_as_float(el.y);
-            const float key = has_bias ? __fadd_rn(gate::key_sigmoidf(l), __ldg(bias + e)) : l;
-            hi = gate::ordered_key(key);
-            lo = ~static_cast<uint32_t>(e);
-        }
-        // k rounds: the largest key, ties to the lower expert index; the winner keeps its rank
-        int rank = k;
-        for (int j = 0; j < k; ++j) {
-            const uint32_t m = __reduce_max_sync(kFullMask, hi);
-            const uint32_t win = __reduce_max_sync(kFullMask, hi == m ? lo : 0u);
-            if (hi == m && lo == win) {
-                rank = j;
-                hi = 0;
+            if (!sigmoid) {
+                gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane,
+                                        topk_idx + t * k, topk_w + t * k);
+                continue;
+            }
+            if (lane < k) {
+                cand.by_rank[slot * k + lane] = my_e;
+                cand.l_by_rank[slot * k + lane] = row[my_e];
+            }
+        } else {
+            // the candidates are captured: start the next token's loads
+            if (t + 1 < t_end) prefetch_row<EPL>(row + E, E, lane, lg);
+            // exact keys of the candidates, one per lane
+            int e = 0;
+            float l = 0.0f;
+            uint32_t hi = 0, lo = 0;
+            if (lane < C) {
+                const uint2 el = cand.el[lane];
+                e = static_cast<int>(el.x);
+                l = __uint_as_float(el.y);
+                const float key = has_bias ? __fadd_rn(gate::key_sigmoidf(l), __ldg(bias + e)) : l;
+                hi = gate::ordered_key(key);
+                lo = ~static_cast<uint32_t>(e);
+            }
+            // k rounds: the largest key, ties to the lower expert index; the winner keeps its rank
+            int rank = k;
+            const uint32_t top = __reduce_max_sync(kFullMask, hi);
+            const uint32_t bottom = __reduce_min_sync(kFullMask, lane < C ? hi : 0xFFFFFFFFu);
+            if (top - bottom < (1u << 26)) {
+                // one reduction per round: the key's offset above the lowest candidate key and the
+                // lane (candidates sit in ascending expert order, so a lower lane is a lower
+                // index) packed into one word that orders like (key, -index); 0 marks "taken"
+                uint32_t p = lane < C ? ((hi - bottom + 1u) << 5) | static_cast<uint32_t>(31 - lane) : 0u;
+                for (int j = 0; j < k; ++j) {
+                    if (p == __reduce_max_sync(kFullMask, p)) {
+                        rank = j;
+                        p = 0;
+                    }
+                }
+            } else {
+                for (int j = 0; j < k; ++j) {
+                    const uint32_t m = __reduce_max_sync(kFullMask, hi);
+                    const uint32_t win = __reduce_max_sync(kFullMask, hi == m ? lo : 0u);
+                    if (hi == m && lo == win) {
+                        rank = j;
+                        hi = 0;
+                    }
+                }
+            }
+            const bool chosen = rank < k;
+            if (!sigmoid) {  // softmax weights need the whole row: lane j takes the j-th expert
+                if (chosen) cand.by_rank[rank] = e;
+                __syncwarp();
+                const int my_e = lane < k ? cand.by_rank[lane] : 0;
+                gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane,
+                                        topk_idx + t * k, topk_w + t * k);
+                continue;
+            }
+            if (chosen) {
+                cand.by_rank[slot * k + rank] = e;
+                cand.l_by_rank[slot * k + rank] = l;
             }
         }
-        const bool chosen = rank < k;
-        if (!sigmoid) {  // softmax weights need the whole row: lane j takes the j-th expert
-            if (chosen) cand.by_rank[rank] = e;
-            __syncwarp();
-            const int my_e = lane < k ? cand.by_rank[lane] : 0;
-            gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane, idx_out, w_out);
-            continue;
-        }
-        // weights in fp64, rounded once to fp32 (the correctly rounded values of s_j / sum s,
-        // except in rare halfway cases), so the reduce that uses them is reproducible too
-        const double sd = chosen ? 1.0 / (1.0 + exp(-static_cast<double>(l))) : 0.0;
-        double denom = sd;
-        if (renormalize) {
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) denom += __shfl_xor_sync(kFullMask, denom, off);
-        }
-        if (chosen) {
-            const float w = !renormalize ? static_cast<float>(sd)
-                                         : (denom == 0.0 ? 0.0f : static_cast<float>(sd / denom));
-            idx_out[rank] = e;
-            w_out[rank] = w;
+        if (slot + 1 == batch || t + 1 == t_end) {
+            gate::write_batch(cand, slot + 1, k, renormalize, lane, topk_idx + t_batch * k,
+                              topk_w + t_batch * k);
+            t_batch = t + 1;
         }
     }
 }
 
-template <int EPL>
+template <int EPL, bool kFull>
 cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, int k, int score_fn,
                         int renormalize, int32_t* idx, float* w, cudaStream_t s) {
     // one wave: as many warps as fit on the GPU at once, each taking a run of consecutive tokens
@@ -199,7 +218,7 @@ cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, in
     int resident_warps = resident[dev].load(std::memory_order_acquire);
     if (resident_warps == 0) {
         int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gate_topk_kernel<EPL>,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gate_topk_kernel<EPL, kFull>,
                                                           kGateWarps * 32, 0) != cudaSuccess || per_sm < 1)
             per_sm = 1;
         resident_warps = per_sm * kGateWarps * num_sms();
@@ -207,8 +226,16 @@ cudaError_t launch_gate(const float* logits, const float* bias, int T, int E, in
     }
     const int warps = min(T, resident_warps);
     const dim3 grid((warps + kGateWarps - 1) / kGateWarps);
-    return launch_pdl(gate_topk_kernel<EPL>, grid, dim3(kGateWarps * 32), 0, s, logits, bias, T, E,
+    return launch_pdl(gate_topk_kernel<EPL, kFull>, grid, dim3(kGateWarps * 32), 0, s, logits, bias, T, E,
                       k, score_fn, renormalize, warps, idx, w);
+}
+
+template <int EPL>
+cudaError_t launch_gate_epl(const float* logits, const float* bias, int T, int E, int k, int score_fn,
+                            int renormalize, int32_t* idx, float* w, cudaStream_t s) {
+    if (E == 32 * EPL)
+        return launch_gate<EPL, true>(logits, bias, T, E, k, score_fn, renormalize, idx, w, s);
+    return launch_gate<EPL, false>(logits, bias, T, E, k, score_fn, renormalize, idx, w, s);
 }
 
 // Largest |approx_sigmoidf(l) - key_sigmoidf(l)| over the finite fp32 l with |l| <= 2^7: the
@@ -261,11 +288,11 @@ extern "C" tk_status tk_gate_topk(const float* logits, const float* bias, int T,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int epl = (E + 31) / 32;
     cudaError_t err;
-    if (epl <= 1) err = launch_gate<1>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
-    else if (epl <= 2) err = launch_gate<2>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
-    else if (epl <= 4) err = launch_gate<4>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
-    else if (epl <= 8) err = launch_gate<8>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
-    else if (epl <= 16) err = launch_gate<16>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
-    else err = launch_gate<32>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    if (epl <= 1) err = launch_gate_epl<1>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 2) err = launch_gate_epl<2>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 4) err = launch_gate_epl<4>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 8) err = launch_gate_epl<8>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else if (epl <= 16) err = launch_gate_epl<16>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
+    else err = launch_gate_epl<32>(logits, bias, T, E, k, score_fn, renormalize, topk_idx, topk_w, s);
     return check_launch(err, "gate_topk_kernel");
 }
