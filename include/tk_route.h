@@ -364,6 +364,17 @@ TK_API tk_status tk_selftest_bounded_wait(int64_t limit_ns, int32_t* err_flag, v
  */
 TK_API tk_status tk_selftest_gate_margin(float* max_err, void* stream);
 
+/*
+ * Self-test of the load-balance statistics' double-precision scores (no counterpart on the
+ * pages: it checks on the GPU the accuracy of the short path that tk_balance_stats and
+ * tk_balance_score_sums use for arguments of magnitude <= 708 -- a table-driven exponential
+ * and a Newton-refined reciprocal -- against the library's exp and division). For every finite
+ * fp32 l with |l| <= 708 (about 2.3e9 values), writes to max_rel_err[0] the largest relative
+ * difference of e^-l and to max_rel_err[1] that of the logistic score 1/(1 + e^-l) (device
+ * doubles, set to 0 first by this call). Both are expected within a few ulps (2^-50).
+ */
+TK_API tk_status tk_selftest_balance_exp(double* max_rel_err, void* stream);
+
 /* Name of a status code (static string). */
 TK_API const char* tk_status_str(int status);
 

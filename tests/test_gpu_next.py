@@ -44,6 +44,64 @@ def test_balance_stats_empty_batch():
     assert (P == 0).all() and (f == 0).all() and loss.item() == 0.0
 
 
+def _balance_vs_oracle(logits, k, score):
+    logits_d = torch.from_numpy(logits).cuda()
+    idx, _ = tk.gate_topk(logits_d, k, score)
+    rm = tk.route_map(idx, logits.shape[1], 1)
+    P, f, loss = tk.balance_stats(logits_d, rm.counts, k, score)
+    torch.cuda.synchronize()
+    fn = oracle.SOFTMAX if score == "softmax" else oracle.SIGMOID
+    Pr, fr, lr = oracle.balance_stats(logits, rm.counts.cpu().numpy(), k, fn)
+    np.testing.assert_allclose(P.cpu().numpy(), Pr, rtol=ULP32, atol=0, equal_nan=True)
+    np.testing.assert_allclose(f.cpu().numpy(), fr, rtol=ULP32, atol=0)
+    np.testing.assert_allclose(loss.cpu().numpy(), np.float32(lr), rtol=ULP32, atol=0, equal_nan=True)
+    return Pr
+
+
+@pytest.mark.parametrize("score", ["sigmoid", "softmax"])
+def test_balance_stats_extreme_logits(score):
+    """Scores computed on both sides of the statistics' short double-precision path (magnitudes
+    up to 708) and on the library path beyond: rows scaled to 300, 707.9, 708, 708.1, 750, 1e4
+    and 1e30, the boundary values themselves, and infinite logits (-inf only for softmax, where
+    +inf makes the row's maximum infinite)."""
+    rng = np.random.default_rng(31 + (score == "softmax"))
+    T, E, k = 900, 96, 6
+    scale = rng.choice([1.0, 300.0, 707.9, 708.0, 708.1, 750.0, 1e4, 1e30], size=(T, 1))
+    logits = (rng.standard_normal((T, E)) * scale).astype(np.float32)
+    pick = rng.random((T, E))
+    logits[pick < 0.02] = np.float32(708.0)
+    logits[(pick >= 0.02) & (pick < 0.04)] = np.float32(-708.0)
+    logits[(pick >= 0.04) & (pick < 0.05)] = np.nextafter(np.float32(708.0), np.float32(np.inf))
+    logits[(pick >= 0.05) & (pick < 0.06)] = -np.inf
+    if score == "sigmoid":
+        logits[(pick >= 0.06) & (pick < 0.07)] = np.inf
+    Pr = _balance_vs_oracle(logits, k, score)
+    assert np.isfinite(Pr).all()
+
+
+def test_balance_stats_non_finite_rows():
+    """A NaN logit makes its token's normalised scores NaN (so every P), and a sigmoid row whose
+    scores all underflow to 0 divides 0 by 0: both sides give NaN in the same places."""
+    rng = np.random.default_rng(33)
+    logits = rng.standard_normal((300, 64)).astype(np.float32)
+    logits[17, 5] = np.nan
+    _balance_vs_oracle(logits, 4, "sigmoid")
+    _balance_vs_oracle(logits, 4, "softmax")
+    logits = rng.standard_normal((300, 64)).astype(np.float32)
+    logits[40, :] = -800.0
+    assert np.isnan(_balance_vs_oracle(logits, 4, "sigmoid")).all()
+
+
+def test_balance_short_path_accuracy():
+    """Exhaustively over every fp32 logit with |l| <= 708: the statistics' table-driven e^-l and
+    Newton-refined logistic score stay within 2^-50 relative of the library's exp and division."""
+    err = tk.selftest_balance_exp()
+    torch.cuda.synchronize()
+    e_exp, e_sig = (float(v) for v in err.cpu())
+    print(f"largest relative difference: exp {e_exp:.3e}, logistic {e_sig:.3e}")
+    assert e_exp < 2.0 ** -50 and e_sig < 2.0 ** -50
+
+
 @pytest.mark.parametrize("wl", [W.MID, W.V3.with_(T=3000), *LARGE_E], ids=lambda w: w.name)
 def test_balance_sums_then_finalize_is_the_one_call(wl):
     logits, bias = W.gate_inputs(wl, "cuda")

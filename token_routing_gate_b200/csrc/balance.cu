@@ -8,7 +8,9 @@
 //     E > 256, to bound registers). Each lane holds experts lane, lane+32, ... of a token,
 //     normalises their unbiased scores over the row (warp reductions) and adds them into
 //     per-lane double accumulators, loading the next token's logits meanwhile; the CTA then
-//     sums its warps in order and writes one row of a [tiles x E] partial-sum matrix.
+//     sums its warps in order and writes one row of a [tiles x E] partial-sum matrix. Up to
+//     256 experts, the scores' exponentials and reciprocals take a short double-precision path
+//     (below) for arguments of magnitude <= 708 and the library's exp and division beyond.
 //   balance_final_kernel: one CTA sums each column (up to 8 threads per column, each over a
 //     contiguous range of tiles with 16 loads in flight, the range sums then added in order),
 //     forms P, f and the loss with a fixed-order tree. The grouping depends on T and E only, so
@@ -45,6 +47,75 @@ __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFullMask, v, off));
     return v;
+}
+
+// Double-precision e^x for |x| <= kFastExpLimit by Tang's table-driven method (P. T. P. Tang,
+// "Table-driven implementation of the exponential function in IEEE floating-point arithmetic",
+// ACM TOMS 15(2), 1989): x = (32 m + j) ln2/32 + r with |r| <= ln2/64, so
+// e^x = 2^m * 2^(j/32) * e^r; e^r - 1 is its Taylor polynomial of degree 6 (the omitted terms
+// are below 2^-60 relative), 2^(j/32) comes from a 32-entry table, and 2^m is added to the
+// exponent field (the result stays a normal number in this range). n = 32 m + j is x * 32/ln2
+// rounded to the nearest integer by adding and subtracting 1.5 * 2^52; ln2/32 is split into a
+// 37-bit head, whose product with |n| < 2^16 is exact, and a tail.
+constexpr double kFastExpLimit = 708.0;
+
+__device__ __forceinline__ double exp_table_driven(double x, const double* __restrict__ two_j32) {
+    constexpr double kShift = 0x1.8p52;                 // 1.5 * 2^52
+    constexpr double k32OverLn2 = 0x1.71547652b82fep+5;  // 32 / ln2
+    constexpr double kLn2Over32Hi = 0x1.62e42fefa0000p-6;
+    constexpr double kLn2Over32Lo = 0x1.cf79abc9e3b3ap-45;
+    const double shifted = fma(x, k32OverLn2, kShift);
+    const int n = __double2loint(shifted);              // the rounded x * 32/ln2, two's complement
+    const double nd = shifted - kShift;
+    double r = fma(-nd, kLn2Over32Hi, x);
+    r = fma(-nd, kLn2Over32Lo, r);
+    double p = 1.0 / 720.0;
+    p = fma(p, r, 1.0 / 120.0);
+    p = fma(p, r, 1.0 / 24.0);
+    p = fma(p, r, 1.0 / 6.0);
+    p = fma(p, r, 0.5);
+    p = fma(p, r, 1.0);
+    p *= r;                                              // e^r - 1
+    const double t = two_j32[n & 31];
+    const double y = fma(t, p, t);                       // 2^(j/32) e^r, in [0.98, 2.03)
+    const int exponent_add = static_cast<int>(static_cast<uint32_t>(n >> 5) << 20);  // 2^m
+    return __hiloint2double(__double2hiint(y) + exponent_add, __double2loint(y));
+}
+
+// 1/d for d >= 1 of moderate size: the hardware approximation refined by two Newton-Raphson
+// steps y <- y + y (1 - d y), each of which squares the relative error.
+__device__ __forceinline__ double reciprocal_newton(double d) {
+    double y;
+    asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(d));
+    y = fma(y, fma(-d, y, 1.0), y);
+    return fma(y, fma(-d, y, 1.0), y);
+}
+
+// The unbiased logistic score 1/(1 + e^-l) and the softmax numerator e^x (x = l - max <= 0).
+// The short path takes its argument clamped to the fast range, so it is safe (and branch-free,
+// letting a lane's experts interleave) for any input; in_short_range says whether its result
+// stands, else the library form below replaces it.
+__device__ __forceinline__ bool logistic_in_short_range(float l) {
+    return fabsf(l) <= static_cast<float>(kFastExpLimit);  // false for NaN
+}
+__device__ __forceinline__ double logistic_short(float l, const double* __restrict__ two_j32) {
+    const double x = fmin(fmax(-static_cast<double>(l), -kFastExpLimit), kFastExpLimit);
+    return reciprocal_newton(1.0 + exp_table_driven(x, two_j32));
+}
+__device__ __forceinline__ double logistic_library(float l) {
+    return 1.0 / (1.0 + exp(-static_cast<double>(l)));
+}
+__device__ __forceinline__ double logistic_score(float l, const double* __restrict__ two_j32) {
+    return logistic_in_short_range(l) ? logistic_short(l, two_j32) : logistic_library(l);
+}
+__device__ __forceinline__ bool numerator_in_short_range(double x) { return x >= -kFastExpLimit; }
+__device__ __forceinline__ double numerator_short(double x, const double* __restrict__ two_j32) {
+    return exp_table_driven(fmin(fmax(x, -kFastExpLimit), 0.0), two_j32);
+}
+
+// Fills the 2^(j/32) table of a CTA (the library's exp2, within an ulp); the caller syncs.
+__device__ __forceinline__ void fill_two_j32(double* two_j32) {
+    if (threadIdx.x < 32) two_j32[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) / 32.0);
 }
 
 // One token's logits, lane-strided (experts lane, lane+32, ...); -inf past E or past T.
@@ -107,6 +178,11 @@ __device__ __forceinline__ void column_sums(const double* __restrict__ partial, 
     __syncthreads();
 }
 
+// The short path for up to 8 experts per lane: its branch-free form interleaves a lane's experts,
+// which at 16 or 32 experts per lane would spill; those forms call the library per expert.
+template <int EPL>
+constexpr bool kShortPath = EPL <= 8;
+
 template <int EPL>
 __global__ void __launch_bounds__(stat_warps<EPL>() * 32, EPL == 16 ? 2 : 1)
 balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score_fn,
@@ -114,6 +190,9 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
     constexpr int kStatWarps = stat_warps<EPL>();
     constexpr int kStatTokensPerWarp = kStatTileTokens / kStatWarps;
     extern __shared__ double wsum[];  // [kStatWarps][E]
+    __shared__ double two_j32[32];
+    fill_two_j32(two_j32);
+    __syncthreads();
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -137,19 +216,48 @@ balance_partial_kernel(const float* __restrict__ logits, int T, int E, int score
 #pragma unroll
             for (int i = 0; i < EPL; ++i) m = fmaxf(m, l[i]);
             m = warp_max_f(m);
+            if constexpr (kShortPath<EPL>) {
+                bool slow = false;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int e = i * 32 + lane;
-                s[i] = e < E ? exp(static_cast<double>(l[i]) - static_cast<double>(m)) : 0.0;
-                z += s[i];
+                for (int i = 0; i < EPL; ++i) {
+                    const double x = static_cast<double>(l[i]) - static_cast<double>(m);
+                    s[i] = numerator_short(x, two_j32);
+                    slow = slow || (i * 32 + lane < E && !numerator_in_short_range(x));
+                }
+                if (__any_sync(kFullMask, slow)) {
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i) {
+                        const double x = static_cast<double>(l[i]) - static_cast<double>(m);
+                        if (!numerator_in_short_range(x)) s[i] = exp(x);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i)
+                    s[i] = i * 32 + lane < E ? exp(static_cast<double>(l[i]) - static_cast<double>(m)) : 0.0;
             }
         } else {
+            if constexpr (kShortPath<EPL>) {
+                bool slow = false;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int e = i * 32 + lane;
-                s[i] = e < E ? 1.0 / (1.0 + exp(-static_cast<double>(l[i]))) : 0.0;
-                z += s[i];
+                for (int i = 0; i < EPL; ++i) {
+                    s[i] = logistic_short(l[i], two_j32);
+                    slow = slow || (i * 32 + lane < E && !logistic_in_short_range(l[i]));
+                }
+                if (__any_sync(kFullMask, slow)) {
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i)
+                        if (!logistic_in_short_range(l[i])) s[i] = logistic_library(l[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) s[i] = i * 32 + lane < E ? logistic_library(l[i]) : 0.0;
             }
+        }
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            if (kShortPath<EPL> && i * 32 + lane >= E) s[i] = 0.0;
+            z += s[i];
         }
         const double rz = 1.0 / warp_sum_d(z);
 #pragma unroll
@@ -225,6 +333,39 @@ cudaError_t launch_partial(const float* logits, int T, int E, int score_fn, doub
     }
     return launch_pdl(balance_partial_kernel<EPL>, dim3(tiles), dim3(kStatWarps * 32), smem, s,
                       logits, T, E, score_fn, partial);
+}
+
+// Largest relative differences, over every finite fp32 l with |l| <= kFastExpLimit, between the
+// short path and the library: [0] e^-l (which covers e^x for the softmax numerators, x = -l),
+// [1] the logistic score 1/(1 + e^-l). Positive doubles order like their bit patterns.
+__global__ void __launch_bounds__(256) balance_exp_check_kernel(unsigned long long* max_rel_bits) {
+    __shared__ double two_j32[32];
+    fill_two_j32(two_j32);
+    __syncthreads();
+    const uint32_t limit = __float_as_uint(static_cast<float>(kFastExpLimit)) + 1u;  // bit patterns of [0, 708]
+    const uint64_t n = 2ull * limit;
+    double worst_exp = 0.0, worst_sig = 0.0;
+    for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+        const uint32_t mag = static_cast<uint32_t>(i >> 1);
+        const float l = __uint_as_float(mag | (static_cast<uint32_t>(i & 1) << 31));
+        const double ref_e = exp(-static_cast<double>(l));
+        const double ref_s = 1.0 / (1.0 + ref_e);
+        const double e = exp_table_driven(-static_cast<double>(l), two_j32);
+        const double sg = logistic_score(l, two_j32);
+        worst_exp = fmax(worst_exp, fabs(e - ref_e) / ref_e);
+        worst_sig = fmax(worst_sig, fabs(sg - ref_s) / ref_s);
+    }
+    unsigned long long be = __double_as_longlong(worst_exp), bs = __double_as_longlong(worst_sig);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        be = max(be, __shfl_xor_sync(kFullMask, be, off));
+        bs = max(bs, __shfl_xor_sync(kFullMask, bs, off));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicMax(max_rel_bits, be);
+        atomicMax(max_rel_bits + 1, bs);
+    }
 }
 
 __global__ void tp_mask_kernel(const int32_t* __restrict__ in, int64_t n, int lo, int el,
@@ -333,6 +474,17 @@ extern "C" tk_status tk_balance_finalize(const double* sums, const int32_t* coun
                                      static_cast<cudaStream_t>(stream), sums, 1, counts, T, E, k, P,
                                      f, loss);
     return check_launch(e, "balance_final_kernel");
+}
+
+extern "C" tk_status tk_selftest_balance_exp(double* max_rel_err, void* stream) {
+    using namespace tk;
+    if (max_rel_err == nullptr) return fail_arg("tk_selftest_balance_exp: max_rel_err must not be NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaMemsetAsync(max_rel_err, 0, 2 * sizeof(double), s);
+    if (err != cudaSuccess) return check_launch(err, "tk_selftest_balance_exp: cudaMemsetAsync");
+    balance_exp_check_kernel<<<num_sms() * 8, 256, 0, s>>>(
+        reinterpret_cast<unsigned long long*>(max_rel_err));
+    return check_launch(cudaGetLastError(), "balance_exp_check_kernel");
 }
 
 extern "C" tk_status tk_tp_mask(const int32_t* topk_idx, int T, int k, int E, int tp_size,

@@ -34,7 +34,7 @@ ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "t
                "tk_balance_stats", "tk_balance_score_sums", "tk_balance_finalize", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
                "tk_reduce_backward", "tk_expand_backward", "tk_ep_layout_workspace_bytes",
                "tk_ep_layout", "tk_ep_dispatch", "tk_ep_combine", "tk_selftest_bounded_wait",
-               "tk_selftest_gate_margin",
+               "tk_selftest_gate_margin", "tk_selftest_balance_exp",
                "tk_status_str", "tk_last_error_detail", "tk_abi_version")
 
 
@@ -105,6 +105,8 @@ def _load():
     L.tk_selftest_bounded_wait.restype = i32
     L.tk_selftest_gate_margin.argtypes = [vp, vp]
     L.tk_selftest_gate_margin.restype = i32
+    L.tk_selftest_balance_exp.argtypes = [vp, vp]
+    L.tk_selftest_balance_exp.restype = i32
     L.tk_status_str.argtypes = [i32]
     L.tk_status_str.restype = ctypes.c_char_p
     L.tk_last_error_detail.argtypes = []
@@ -362,6 +364,17 @@ def selftest_gate_margin(max_err=None, stream=None):
     _check("tk_selftest_gate_margin", lib.tk_selftest_gate_margin(_ptr(max_err, F32, 1, "max_err"),
                                                                   _stream(stream)))
     return max_err
+
+
+def selftest_balance_exp(max_rel_err=None, stream=None):
+    """Largest relative differences between the balance statistics' short double-precision path
+    and the library over every finite fp32 l with |l| <= 708: [e^-l, 1/(1 + e^-l)], as a device
+    double tensor [2]."""
+    if max_rel_err is None:
+        max_rel_err = torch.empty(2, dtype=torch.float64, device="cuda")
+    _check("tk_selftest_balance_exp", lib.tk_selftest_balance_exp(
+        _ptr(max_rel_err, F64, 2, "max_rel_err"), _stream(stream)))
+    return max_rel_err
 
 
 # ---------------------------------------------------------------- expert-parallel dispatch / combine
