@@ -27,6 +27,7 @@
 // Every wait is bounded (1 s); a timeout flags TK_DEVERR_TIMEOUT and ends the CTA's loop.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <type_traits>
 #include <stdint.h>
 
 #include "tk_device.cuh"
@@ -47,6 +48,9 @@ namespace {
 #define TK_REDUCE_STAGE_KB 32
 #endif
 
+#ifndef TK_REDUCE_DENSE_CTAS_PER_SM  // resident CTAs per SM of the dense reduce (0: as many as fit)
+#define TK_REDUCE_DENSE_CTAS_PER_SM 5
+#endif
 #ifndef TK_REDUCE_MASKED_VECS_PER_THREAD
 #define TK_REDUCE_MASKED_VECS_PER_THREAD 2
 #endif
@@ -386,6 +390,10 @@ cudaError_t launch_shape(int k, LaunchShape& out) {
         int per_sm = 0;
         err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_kernel<Rows, kStep, kVecs>, kRedThreads, smem);
         if (err != cudaSuccess) return err;
+        if constexpr (std::is_same<Rows, SlotRows>::value && !kStep) {
+            if (TK_REDUCE_DENSE_CTAS_PER_SM > 0 && per_sm > TK_REDUCE_DENSE_CTAS_PER_SM)
+                per_sm = TK_REDUCE_DENSE_CTAS_PER_SM;
+        }
         shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
         shapes[dev][k].ring = ring;
         ready[dev][k].store(true, std::memory_order_release);
