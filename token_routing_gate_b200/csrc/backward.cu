@@ -36,6 +36,9 @@ constexpr int kChunkBytes = kChunkCh * 2;
 constexpr int kStageBudget = TK_BACKWARD_STAGE_KB * 1024;
 constexpr int kRegRows = 8;  // up to this k, per-thread register accumulators for d_w
 
+#ifndef TK_BACKWARD_CTAS_PER_SM  // resident CTAs per SM at most (0: as many as fit)
+#define TK_BACKWARD_CTAS_PER_SM 3
+#endif
 #ifndef TK_BACKWARD_LOAD_POLICY   // L2 policy of the row loads: 0 none, 1 evict-normal, 2 evict-first
 #define TK_BACKWARD_LOAD_POLICY 1
 #endif
@@ -292,6 +295,9 @@ cudaError_t launch_shape(int k, Shape& out) {
         int per_sm = 0;
         err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_backward_kernel, kBwdThreads, smem);
         if (err != cudaSuccess) return err;
+        // Launched after a kernel that leaves L2 full of dirty lines (its own previous call, or
+        // any write-heavy step), 3 CTAs per SM measured 1-2 % faster than the 5 that fit.
+        if (TK_BACKWARD_CTAS_PER_SM > 0 && per_sm > TK_BACKWARD_CTAS_PER_SM) per_sm = TK_BACKWARD_CTAS_PER_SM;
         shapes[dev][k].S = S;
         shapes[dev][k].grid_cap = num_sms() * (per_sm < 1 ? 1 : per_sm);
         ready[dev][k].store(true, std::memory_order_release);
