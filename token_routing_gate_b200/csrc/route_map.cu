@@ -313,14 +313,85 @@ route_scan_kernel(int32_t* __restrict__ tile_counts, int tiles, int stride, int 
     if (threadIdx.x == 0) offsets[E] = carry;
 }
 
+// Many CTAs, for count matrices too large for the fused kernel: G = threads per expert row (a
+// power of two <= 32, so a row's threads sit in one warp), kRouteThreads / G rows per CTA. A
+// thread owns `seg` consecutive 16-byte vectors of its row: it sums them, the row's G threads
+// exclusive-scan their sums with shuffles, and the thread rewrites its vectors as exclusive
+// per-tile prefixes (in place; the padding past the last tile is zero, written by the count
+// kernel, so whole vectors are summed). counts[e] gets the row total. The expert offsets are
+// formed by the scatter kernel from counts.
+struct RowScanShape {
+    int G, seg, grid;
+};
+inline RowScanShape row_scan_shape(int stride, int E) {
+    const int n4 = stride / 4;
+    int G = 1;
+    while (G < 32 && G * kRowBatch < n4) G *= 2;
+    const int rows_per_cta = kRouteThreads / G;
+    return {G, (n4 + G - 1) / G, (E + rows_per_cta - 1) / rows_per_cta};
+}
+
 __global__ void __launch_bounds__(kRouteThreads)
-route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+route_row_scan_kernel(int32_t* __restrict__ tile_counts, int stride, int E, int G, int seg,
+                      int32_t* __restrict__ counts) {
+    pdl_wait();
+    const int rows_per_cta = kRouteThreads / G;
+    const int e = blockIdx.x * rows_per_cta + static_cast<int>(threadIdx.x) / G;
+    const int part = static_cast<int>(threadIdx.x) % G;
+    const int n4 = stride / 4;
+    const int v0 = part * seg;
+    const int v1 = min(n4, v0 + seg);
+    int4* r4 = reinterpret_cast<int4*>(tile_counts + static_cast<int64_t>(e < E ? e : 0) * stride);
+    int32_t mine = 0;
+    if (e < E) {
+        for (int c0 = v0; c0 < v1; c0 += kRowBatch) {
+            int4 v[kRowBatch];
+#pragma unroll
+            for (int i = 0; i < kRowBatch; ++i) v[i] = c0 + i < v1 ? r4[c0 + i] : make_int4(0, 0, 0, 0);
+#pragma unroll
+            for (int i = 0; i < kRowBatch; ++i) mine += v[i].x + v[i].y + v[i].z + v[i].w;
+        }
+    }
+    // exclusive scan of the parts' sums over the row's G lanes (aligned groups within a warp)
+    int32_t incl = mine;
+    for (int off = 1; off < G; off <<= 1) {
+        const int32_t u = __shfl_up_sync(kFullMask, incl, off, G);
+        if (part >= off) incl += u;
+    }
+    const int32_t total = __shfl_sync(kFullMask, incl, G - 1, G);
+    if (e >= E) return;
+    int32_t run = incl - mine;
+    for (int c0 = v0; c0 < v1; c0 += kRowBatch) {
+        int4 v[kRowBatch];
+#pragma unroll
+        for (int i = 0; i < kRowBatch; ++i) v[i] = c0 + i < v1 ? r4[c0 + i] : make_int4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < kRowBatch; ++i) {
+            if (c0 + i >= v1) break;
+            int4 o;
+            o.x = run; run += v[i].x;
+            o.y = run; run += v[i].y;
+            o.z = run; run += v[i].z;
+            o.w = run; run += v[i].w;
+            r4[c0 + i] = o;
+        }
+    }
+    if (part == 0) counts[e] = total;
+}
+
+// One CTA per tile: forms the expert offsets from counts itself (CTA 0 also writes them out),
+// then ranks and scatters the tile's pairs like the fused kernel.
+__global__ void __launch_bounds__(kRouteThreads)
+route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int align,
                      const int32_t* __restrict__ tile_prefix, int stride,
-                     const int32_t* __restrict__ offsets, int32_t* __restrict__ slot_of,
-                     int32_t* __restrict__ token_of, int32_t* err_flag) {
+                     const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                     int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
+                     int32_t* err_flag) {
     extern __shared__ uint32_t smem[];
     uint32_t* bitmap = smem;                                          // [E][kTileWords]
     int32_t* base = reinterpret_cast<int32_t*>(smem + E * kTileWords);  // [E]
+    int32_t* total = base + E;                                        // [E]
+    __shared__ int32_t warp_tot[kRouteThreads / 32];
     pdl_wait();
     const int tile = blockIdx.x;
     const int t0 = tile * kTileTokens;
@@ -332,10 +403,40 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     __syncthreads();
     tile_mark(bitmap, e_reg, n, divk, E, err_flag);
-    for (int e = threadIdx.x; e < E; e += kRouteThreads)
-        base[e] = offsets[e] + tile_prefix[static_cast<int64_t>(e) * stride + tile];
+    for (int e = threadIdx.x; e < E; e += kRouteThreads) total[e] = counts[e];
+    __syncthreads();
+    const int32_t R = cta_padded_scan(total, E, align, base, warp_tot);
+    for (int e = threadIdx.x; e < E; e += kRouteThreads) {
+        if (tile == 0) offsets[e] = base[e];
+        base[e] += tile_prefix[static_cast<int64_t>(e) * stride + tile];
+    }
+    if (tile == 0 && threadIdx.x == 0) offsets[E] = R;
     __syncthreads();
     tile_scatter(bitmap, base, e_reg, n, divk, p0, t0, E, slot_of, token_of);
+}
+
+// The scan and scatter of a count matrix too large for the fused kernel (and of every matrix
+// in the allocation-free entry point). With no tile the single-CTA scan writes the (zero)
+// counts and offsets.
+cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int k, int align,
+                                     int32_t* tile_counts, int tiles, int stride, int32_t* counts,
+                                     int32_t* offsets, int32_t* slot_of, int32_t* token_of,
+                                     int32_t* err_flag, cudaStream_t s, const char** what) {
+    if (tiles == 0) {
+        *what = "route_scan_kernel";
+        return launch_pdl(route_scan_kernel, dim3(1), dim3(scan_threads(E)), 0, s, tile_counts, tiles,
+                          stride, E, align, counts, offsets);
+    }
+    const RowScanShape rs = row_scan_shape(stride, E);
+    *what = "route_row_scan_kernel";
+    cudaError_t err = launch_pdl(route_row_scan_kernel, dim3(rs.grid), dim3(kRouteThreads), 0, s,
+                                 tile_counts, stride, E, rs.G, rs.seg, counts);
+    if (err != cudaSuccess) return err;
+    *what = "route_scatter_kernel";
+    const size_t smem = static_cast<size_t>(E) * (kTileWords + 2) * sizeof(uint32_t);
+    return launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
+                      T, E, k, align, static_cast<const int32_t*>(tile_counts), stride,
+                      static_cast<const int32_t*>(counts), offsets, slot_of, token_of, err_flag);
 }
 
 // Scan and scatter in one kernel, for count matrices of at most kFusedMaxEntries entries: every
@@ -439,17 +540,10 @@ extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, 
                          stride, counts, offsets, slot_of, token_of, err_flag);
         return check_launch(err, "route_scan_scatter_kernel");
     }
-    err = launch_pdl(route_scan_kernel, dim3(1), dim3(scan_threads(E)), 0, s, tile_counts, tiles,
-                     stride, E, align, counts, offsets);
-    if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
-    if (tiles > 0) {
-        const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
-        err = launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
-                         T, E, k, static_cast<const int32_t*>(tile_counts), stride,
-                         static_cast<const int32_t*>(offsets), slot_of, token_of, err_flag);
-        if (err != cudaSuccess) return check_launch(err, "route_scatter_kernel");
-    }
-    return TK_OK;
+    const char* what = "";
+    err = launch_scan_then_scatter(topk_idx, T, E, k, align, tile_counts, tiles, stride, counts,
+                                   offsets, slot_of, token_of, err_flag, s, &what);
+    return check_launch(err, what);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -535,15 +629,8 @@ extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, 
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
                                  tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
-    err = launch_pdl(route_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tile_counts, tiles,
-                     stride, E, align, counts, offsets);
-    if (err != cudaSuccess) return check_launch(err, "route_scan_kernel");
-    if (tiles > 0) {
-        const size_t smem = static_cast<size_t>(E) * (kTileWords + 1) * sizeof(uint32_t);
-        err = launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
-                         T, E, k, static_cast<const int32_t*>(tile_counts), stride,
-                         static_cast<const int32_t*>(offsets), slot_of, token_of, err_flag);
-        if (err != cudaSuccess) return check_launch(err, "route_scatter_kernel");
-    }
-    return TK_OK;
+    const char* what = "";
+    err = launch_scan_then_scatter(topk_idx, T, E, k, align, tile_counts, tiles, stride, counts,
+                                   offsets, slot_of, token_of, err_flag, s, &what);
+    return check_launch(err, what);
 }
