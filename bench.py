@@ -367,9 +367,9 @@ def run_tk(args, wl):
             ev[4].record(stream)
 
     # route map: count + fused scan/scatter while its count matrix (E rows of 128-token tiles,
-    # padded to a multiple of 4) has at most 64K entries, else count, scan and scatter
+    # padded to a multiple of 4) has at most 32K entries, else count, scan and scatter
     tiles = (wl.T + 127) // 128
-    route_launches = 2 if (tiles + 3) // 4 * 4 * wl.E <= 65536 else 3
+    route_launches = 2 if (tiles + 3) // 4 * 4 * wl.E <= 32768 else 3
     launches_per_step = 1 + route_launches + 1 + (1 if wl.align > 1 else 0) + 1
     for _ in range(args.warmup):
         step()

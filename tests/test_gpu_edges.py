@@ -74,7 +74,8 @@ def _rand_inputs(wl, rng, rows=None):
     (5, 32, 32, 128, "sigmoid", True, 1, "fp8"),        # k = E = warp width
     (20000, 24, 3, 64, "sigmoid", True, 1, "bf16"),     # several tokens per gate warp
     (40000, 16, 2, 8, "softmax", False, 4, "bf16"),     # 313 tiles, small count matrix: fused
-    (20000, 512, 4, 8, "sigmoid", True, 4, "bf16"),     # count matrix > 64K: separate scan kernel
+    (20000, 512, 4, 8, "sigmoid", True, 4, "bf16"),     # count matrix > 32K: many-CTA row scan
+    (33000, 256, 8, 8, "sigmoid", True, 1, "bf16"),     # 258 tiles: row scan, 16 threads per row, 3 idle
     (257, 37, 5, 264, "sigmoid", True, 1, "bf16"),      # ragged T, E % 32 != 0, H % 128 != 0
     (300, 1000, 12, 256, "softmax", False, 7, "bf16"),  # E close to the limit, odd alignment
     (64, 1024, 32, 128, "sigmoid", True, 128, "fp8"),   # largest E and k
