@@ -382,7 +382,9 @@ TK_API const char* tk_status_str(int status);
  * thread-local buffer, valid until the next call on that thread). */
 TK_API const char* tk_last_error_detail(void);
 
-/* ABI version of this header: (major << 16) | minor. */
+/* ABI version of this header: (major << 16) | minor. The minor number grows when entry points
+ * are added (1.2: tk_selftest_gate_margin and tk_selftest_balance_exp); the major number would
+ * change only if an existing signature or meaning did. */
 TK_API int tk_abi_version(void);
 
 #ifdef __cplusplus

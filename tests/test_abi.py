@@ -48,6 +48,7 @@ def test_sizes_and_strings(tk):
     assert tk.lib.tk_status_str(0) == b"TK_OK"
     assert tk.lib.tk_status_str(1) == b"TK_ERR_INVALID_ARG"
     assert tk.lib.tk_abi_version() >> 16 == 1
+    assert tk.lib.tk_abi_version() & 0xFFFF >= 2  # the self-test entry points are there
 
 
 FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: the calls fail validation first
