@@ -35,8 +35,11 @@ constexpr int kGateWarps = 8;  // tokens per CTA
 //     group_threshold, then the k-th largest lane maximum when the cheap one leaves more than
 //     32 candidates). The k-th largest exact key is then >= theta - eps, and every expert whose
 //     exact key reaches it has A >= theta - 2 eps. Those experts (the candidates) get their
-//     exact keys, one per lane, and k rounds of two warp reductions select among them exactly
-//     as among all E; each winner keeps its rank and writes its own outputs.
+//     exact keys, one per lane in ascending expert order, and k rounds of warp reductions select
+//     among them exactly as among all E: one reduction per round over (key offset, lane) packed
+//     into a word while the candidates' key images span less than 2^26, else two (the key, then
+//     the lowest index holding it). Each winner records its expert and logit by rank; with
+//     logistic scores the weights of up to 32/k consecutive tokens are then computed together.
 // More than 32 candidates (many equal or nearly equal keys), a non-finite or huge bias, or
 // fewer than k lanes holding an expert send the token down the full path: every exact key, a
 // per-lane sort and k rounds over the sorted lists.
