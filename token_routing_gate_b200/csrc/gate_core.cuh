@@ -237,25 +237,35 @@ __device__ __forceinline__ int select_topk(uint64_t (&v)[EPL], int k, int lane) 
     return my_e;
 }
 
-// Outputs of a batch of n consecutive tokens (n*k <= 32) with logistic scores, whose choices sit
-// in c.by_rank / c.l_by_rank: lane q*k + j takes token q's rank-j choice, computes its unbiased
-// score 1 / (1 + e^-l) in double, adds the k scores of its token in rank order when renormalising
-// (the order of the defining sum), and writes entry q*k + j of the batch's outputs (consecutive
-// in idx_out and w_out), rounded once to fp32. One pass serves up to 32/k tokens, so the double
-// arithmetic runs on up to every lane instead of k of them per token.
-__device__ __forceinline__ void write_batch(const Candidates& c, int n, int k, int renormalize, int lane,
+// Outputs of a batch of n consecutive tokens (n*k <= 32) whose choices sit in c.by_rank /
+// c.l_by_rank: lane q*k + j takes token q's rank-j choice and computes its unbiased score in
+// double -- the logistic value 1 / (1 + e^-l), or for softmax (renormalised only) e^(l - l0)
+// with l0 the token's rank-0 logit, its largest (the full softmax denominator cancels in the
+// renormalisation; an infinite or NaN l0 gives zero weights) -- adds the k scores of its token
+// in rank order when renormalising (the order of the defining sum), and writes entry q*k + j of
+// the batch's outputs (consecutive in idx_out and w_out), rounded once to fp32. One pass serves
+// up to 32/k tokens, so the double arithmetic runs on up to every lane instead of k of them per
+// token.
+__device__ __forceinline__ void write_batch(const Candidates& c, int n, int k, int score_fn,
+                                            int renormalize, int lane,
                                             int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     __syncwarp();  // the batch's choices are in c
     const bool mine = lane < n * k;
+    const int first = lane - lane % k;  // this token's rank-0 lane (mod 32 past the batch)
     double s = 0.0;
     int e = 0;
     if (mine) {
         e = c.by_rank[lane];
-        s = 1.0 / (1.0 + exp(-static_cast<double>(c.l_by_rank[lane])));
+        const float l = c.l_by_rank[lane];
+        if (score_fn == TK_SCORE_SIGMOID) {
+            s = 1.0 / (1.0 + exp(-static_cast<double>(l)));
+        } else {
+            const float l0 = c.l_by_rank[first];
+            if (l0 != -INFINITY && l0 == l0) s = exp(static_cast<double>(l) - static_cast<double>(l0));
+        }
     }
     double denom = 1.0;
     if (renormalize) {
-        const int first = lane - lane % k;  // this token's rank-0 lane (mod 32 past the batch)
         denom = 0.0;
         for (int j = 0; j < k; ++j) denom += __shfl_sync(kFullMask, s, first + j);
     }

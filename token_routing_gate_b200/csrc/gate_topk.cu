@@ -104,7 +104,11 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
     gate::Candidates& cand = cands[threadIdx.x >> 5];
     const bool has_bias = bias != nullptr;
     const bool sigmoid = score_fn == TK_SCORE_SIGMOID;
-    const int batch = sigmoid ? 32 / k : 1;  // tokens per weight pass
+    // weights from the chosen experts alone (logistic scores, or renormalised softmax) are
+    // computed for up to 32/k consecutive tokens at once when the warp routes several; a warp
+    // with one token (and plain softmax, which needs the whole row) writes each token directly
+    const bool batched = (sigmoid || renormalize) && t_end - t_begin > 1;
+    const int batch = batched ? 32 / k : 1;  // tokens per weight pass
 
     float b[EPL];  // this lane's selection biases, shared by all tokens
 #pragma unroll
@@ -141,7 +145,7 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
             gate::build_keys<EPL>(lg, b, has_bias, E, lane, v);
             if (t + 1 < t_end) prefetch_row<EPL>(row + E, E, lane, lg);
             const int my_e = gate::select_topk<EPL>(v, k, lane);
-            if (!sigmoid) {
+            if (!batched) {
                 gate::write_choice<EPL>(row, my_e, E, k, score_fn, renormalize, lane,
                                         topk_idx + t * k, topk_w + t * k);
                 continue;
@@ -191,7 +195,7 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
                 }
             }
             const bool chosen = rank < k;
-            if (!sigmoid) {  // softmax weights need the whole row: lane j takes the j-th expert
+            if (!batched) {  // softmax weights need the whole row: lane j takes the j-th expert
                 if (chosen) cand.by_rank[rank] = e;
                 __syncwarp();
                 const int my_e = lane < k ? cand.by_rank[lane] : 0;
@@ -205,7 +209,7 @@ gate_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bia
             }
         }
         if (slot + 1 == batch || t + 1 == t_end) {
-            gate::write_batch(cand, slot + 1, k, renormalize, lane, topk_idx + t_batch * k,
+            gate::write_batch(cand, slot + 1, k, score_fn, renormalize, lane, topk_idx + t_batch * k,
                               topk_w + t_batch * k);
             t_batch = t + 1;
         }
