@@ -159,18 +159,22 @@ def test_candidate_keys_spanning_many_binades(score):
     _check(logits, bias, k, score)
 
 
+@pytest.mark.parametrize("score", ["sigmoid", "softmax"])
 @pytest.mark.parametrize("renormalize", [True, False])
 @pytest.mark.parametrize("k", [8, 6, 5, 3])
-def test_weight_batches_with_full_path_tokens(k, renormalize):
+def test_weight_batches_with_full_path_tokens(k, renormalize, score):
     """Enough tokens that each warp routes several and computes their weights together (32/k
-    tokens per pass), with every third token sent down the full path (40 equal top keys) in the
-    middle of a batch."""
-    rng = np.random.default_rng(40 + k + renormalize)
+    tokens per pass; logistic scores, or softmax when renormalised), with every third token sent
+    down the full path (40 equal top keys) in the middle of a batch. Plain softmax writes each
+    token's weights from the whole row."""
+    rng = np.random.default_rng(40 + k + renormalize + 10 * (score == "softmax"))
     T, E = 20000, 256
     logits = rng.standard_normal((T, E)).astype(np.float32)
-    bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
     tied = rng.choice(E, 40, replace=False)
-    bias[tied] = 0.05
+    bias = None
+    if score == "sigmoid":
+        bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+        bias[tied] = 0.05
     logits[::3, :] -= 4.0
     logits[::3][:, tied] = 3.0
-    _check(logits, bias, k, "sigmoid", renormalize)
+    _check(logits, bias, k, score, renormalize)
