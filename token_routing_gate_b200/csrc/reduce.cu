@@ -16,10 +16,12 @@
 // The ring holds 32 KB, so a unit whose k = 8 rows are all valid takes 16 KB (two in flight, as a
 // fixed two-stage ring would), while a unit with few valid rows -- a masked route map, an
 // expert-parallel destination's rows -- takes only what it loads and up to 16 units are in
-// flight. About six CTAs fit on an SM (~190 KB of loads in flight). A measured sweep on B200
-// (ring size, chunk width, consumer warps) put this shape at the HBM copy roofline; deeper rings
-// with fewer CTAs per SM were up to 30% slower. The grid is persistent (SM count x CTAs per SM)
-// and CTAs stride over units.
+// flight. Six CTAs fit on an SM; the dense reduce keeps five (160 KB of loads in flight per
+// SM): after a write-heavy kernel (expand in the routing step) five took 171 us at T=8192 where
+// six took 183, while after a read-heavy one six were 4 us faster. A measured sweep on B200
+// (ring size, chunk width, consumer warps) put this shape at the HBM copy roofline; deeper
+// rings with fewer CTAs per SM were up to 30% slower. The grid is persistent (SM count x CTAs
+// per SM) and CTAs stride over units.
 // The row loads carry an explicit L2 evict-normal policy. Measured on B200 at T=8192, H=7168,
 // k=8: with it the reduce after dispatch and the reduce run back to back were both faster than
 // with no policy operand (forward step 366.8 -> 364.9 us; back-to-back reduce 155.5 -> 152.9 us).

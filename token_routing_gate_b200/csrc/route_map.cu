@@ -9,7 +9,9 @@
 //             [E x tiles] count matrix (expert-major, each expert's row padded to a multiple of
 //             4 tiles so that it reads as 16-byte vectors); the grid also fills token_of with -1.
 //   scan    : turns each expert's row into exclusive per-tile prefixes, sums it into
-//             counts[e], rounds it up to the alignment and scans over experts for offsets[].
+//             counts[e], rounds it up to the alignment and scans over experts for offsets[]
+//             (for large matrices the rows are scanned on many CTAs and the scatter kernel
+//             forms the offsets).
 //   scatter : one CTA per tile marks, per expert, which of its tokens chose that expert in a
 //             shared-memory bitmap; a pair's rank inside the tile is the population count of
 //             the bits below its token. slot = offsets[e] + tile prefix[e] + rank -- the same
