@@ -597,11 +597,20 @@ def run_op(args, wl):
         P = (torch.empty(E, device=dev), torch.empty(E, device=dev), torch.empty(1, device=dev))
         ws = tk._workspace(int(tk.lib.tk_balance_stats_workspace_bytes(T, E)), dev)
         masked = torch.empty_like(idx)
+        rm_tp = tk.route_map(masked.zero_(), E // 8, 1)
+        rm_win = tk.route_map_window(idx, E, 3 * (E // 8), E // 8, 1)
         calls = {
             "balance_stats": (lambda: tk.balance_stats(logits, rm.counts, k, wl.score, workspace=ws, out=P,
                                                        stream=stream),
                               T * E * 4 + E * 4 + ((T + 63) // 64) * E * 8 * 2 + 3 * E * 4, 2),
             "tp_mask": (lambda: tk.tp_mask(idx, E, 8, 3, out=masked, stream=stream), T * k * 8, 1),
+            # one tensor-parallel rank's route map (8 ranks): the mask then the route map, and
+            # the window route map doing both in one call
+            "tp_mask_then_route_map": (lambda: (tk.tp_mask(idx, E, 8, 3, out=masked, stream=stream),
+                                                tk.route_map(masked, E // 8, 1, out=rm_tp, stream=stream)),
+                                       T * k * 8 + T * k * 12, 3),
+            "route_map_window": (lambda: tk.route_map_window(idx, E, 3 * (E // 8), E // 8, 1, out=rm_win,
+                                                             stream=stream), T * k * 12, 2),
         }
         metric = "load-balance statistics and TP mask us per call"
     peak, peak_kind = load_peak()

@@ -119,6 +119,26 @@ TK_API tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int 
                        size_t workspace_bytes, int32_t* err_flag, void* stream);
 
 /*
+ * Route map of one window of experts: the tensor-parallel mask (tk_tp_mask) fused into the route
+ * map (147227.xyz "moe/": tensor-parallel mask, next to the token-to-expert mapping). A pair
+ * whose expert lies in [expert_lo, expert_lo + E) is routed to local expert e - expert_lo; every
+ * other pair is masked (slot -1). The outputs are those of tk_tp_mask(tp_size = E_total / E,
+ * tp_rank = expert_lo / E) followed by tk_route_map with E experts, without the masked index
+ * array or the extra launch; unlike that pair of calls, an index outside [0, E_total) other than
+ * -1 sets TK_DEVERR_EXPERT_RANGE.
+ *   E_total   all experts the indices refer to; 0 <= expert_lo and expert_lo + E <= E_total
+ *   E         the window's experts (1 <= E <= 1024): counts [E], offsets [E+1], token_of
+ *             [tk_max_rows(T, E, k, align)] and the workspace (tk_route_map_workspace_bytes(T,
+ *             E, k)) are sized by it
+ * Every other argument as in tk_route_map.
+ */
+TK_API tk_status tk_route_map_window(const int32_t* topk_idx, int T, int E_total, int k,
+                                     int expert_lo, int E, int align, int32_t* counts,
+                                     int32_t* offsets, int32_t* slot_of, int32_t* token_of,
+                                     void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                                     void* stream);
+
+/*
  * Allocation-free form of tk_route_map (the pages have no counterpart: this exists only for
  * callers that cannot allocate device memory, such as a serving engine or plugin host that
  * owns all device memory and hands a component only its inputs and outputs, or a
@@ -383,8 +403,9 @@ TK_API const char* tk_status_str(int status);
 TK_API const char* tk_last_error_detail(void);
 
 /* ABI version of this header: (major << 16) | minor. The minor number grows when entry points
- * are added (1.2: tk_selftest_gate_margin and tk_selftest_balance_exp); the major number would
- * change only if an existing signature or meaning did. */
+ * are added (1.2: tk_selftest_gate_margin and tk_selftest_balance_exp; 1.3:
+ * tk_route_map_window); the major number would change only if an existing signature or meaning
+ * did. */
 TK_API int tk_abi_version(void);
 
 #ifdef __cplusplus

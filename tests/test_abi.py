@@ -48,7 +48,7 @@ def test_sizes_and_strings(tk):
     assert tk.lib.tk_status_str(0) == b"TK_OK"
     assert tk.lib.tk_status_str(1) == b"TK_ERR_INVALID_ARG"
     assert tk.lib.tk_abi_version() >> 16 == 1
-    assert tk.lib.tk_abi_version() & 0xFFFF >= 2  # the self-test entry points are there
+    assert tk.lib.tk_abi_version() & 0xFFFF >= 3  # the self-tests and the window route map are there
 
 
 FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: the calls fail validation first
@@ -259,3 +259,19 @@ def test_product_modules_do_not_reach_the_oracle():
     for name in sorted(os.listdir(csrc)):
         text = open(os.path.join(csrc, name)).read()
         assert "oracle" not in text.lower(), name
+
+
+def test_route_map_window_rejects_bad_windows(tk):
+    L = tk.lib
+    ws = L.tk_route_map_workspace_bytes(128, 32, 8)
+    ok = [FAKE, 128, 256, 8, 64, 32, 1, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None, None]
+    for i, v, what in [(4, -1, "window"), (4, 225, "window"), (5, 0, "E=0"), (5, 257, "window"), (5, 1025, "E=1025"),
+                       (3, 33, "k"), (6, 0, "align"), (12, ws - 16, "workspace"), (7, None, "NULL")]:
+        a = list(ok)
+        a[i] = v
+        assert L.tk_route_map_window(*a) == 1, what
+        detail = L.tk_last_error_detail().decode()
+        assert what in detail and "tk_route_map_window" in detail, detail
+    a = list(ok)
+    a[11] = MISALIGNED
+    assert L.tk_route_map_window(*a) == 1 and "aligned" in L.tk_last_error_detail().decode()

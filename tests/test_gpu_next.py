@@ -223,6 +223,59 @@ def test_tp_mask_then_route(tp):
     np.testing.assert_array_equal(inplace.cpu().numpy(), oracle.tp_mask(idx_h, wl.E, tp, tp - 1))
 
 
+@pytest.mark.parametrize("T,E,k,tp,align", [
+    (3000, 256, 8, 8, 128),    # V3 experts over 8 tensor-parallel ranks
+    (8192, 256, 8, 2, 1),      # the V3 batch, two ranks
+    (40000, 64, 6, 4, 4),      # several tiles per CTA, fused count matrix
+    (20000, 1024, 4, 2, 16),   # 512 local experts: count matrix past the fused limit
+    (77, 37, 5, 1, 3),         # the whole map as one window
+])
+def test_route_map_window_equals_mask_then_route(T, E, k, tp, align):
+    """tk_route_map_window on each rank's expert window gives exactly tk_tp_mask followed by
+    tk_route_map with the local experts (and the oracle's tp_mask + route_map)."""
+    rng = np.random.default_rng(T + E + tp)
+    idx_h = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    if T > 10:
+        idx_h[5, 1] = -1                      # a pair masked before the call
+    idx = torch.from_numpy(idx_h).cuda()
+    el = E // tp
+    for r in range(tp):
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        got = tk.route_map_window(idx, E, r * el, el, align, err_flag=err)
+        ref = tk.route_map(tk.tp_mask(idx, E, tp, r), el, align)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        for a, b in ((got.counts, ref.counts), (got.offsets, ref.offsets), (got.slot_of, ref.slot_of),
+                     (got.token_of, ref.token_of)):
+            assert torch.equal(a, b)
+        counts, offsets, slot_of, token_of, rc = oracle.route_map(oracle.tp_mask(idx_h, E, tp, r), el, align)
+        assert rc == 0
+        np.testing.assert_array_equal(got.slot_of.cpu().numpy(), slot_of)
+        np.testing.assert_array_equal(got.offsets.cpu().numpy(), offsets)
+        np.testing.assert_array_equal(got.token_of.cpu().numpy(), token_of)
+
+
+def test_route_map_window_flags_indices_outside_all_experts():
+    """An index outside [0, E_total) other than -1 sets the expert-range bit and is masked; one
+    outside the window but inside [0, E_total) is only masked."""
+    T, E, k = 600, 64, 4
+    rng = np.random.default_rng(9)
+    idx_h = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    idx_h[3, 0], idx_h[4, 2] = E, -5
+    idx = torch.from_numpy(idx_h).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = tk.route_map_window(idx, E, 16, 16, 1, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() & 1                     # TK_DEVERR_EXPERT_RANGE
+    slots = got.slot_of.cpu().numpy()
+    assert slots[3, 0] == -1 and slots[4, 2] == -1
+    clean = idx_h.copy()
+    clean[3, 0], clean[4, 2] = -1, -1
+    counts, offsets, slot_of, token_of, _ = oracle.route_map(oracle.tp_mask(clean, E, 4, 1), 16, 1)
+    np.testing.assert_array_equal(slots, slot_of)
+    np.testing.assert_array_equal(got.counts.cpu().numpy(), counts)
+
+
 @pytest.mark.parametrize("T,E,k,H,align,weighted", [
     (300, 16, 4, 264, 8, True),      # ragged chunk, padding rows
     (2048, 256, 8, 7168, 1, True),   # DeepSeek-V3 row shape

@@ -95,4 +95,4 @@ extern "C" const char* tk_status_str(int status) {
 
 extern "C" const char* tk_last_error_detail(void) { return tk::g_detail; }
 
-extern "C" int tk_abi_version(void) { return (1 << 16) | 2; }
+extern "C" int tk_abi_version(void) { return (1 << 16) | 3; }

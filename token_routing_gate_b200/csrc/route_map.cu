@@ -63,8 +63,15 @@ __device__ __forceinline__ int pairs_of_thread(int n) {
     return n > static_cast<int>(threadIdx.x) ? (n - 1 - static_cast<int>(threadIdx.x)) / kRouteThreads + 1 : 0;
 }
 
+// The local expert of a pair's index: raw - lo inside the window [lo, lo + E), else -1
+// (masked). The whole map is the window lo = 0, E = all experts.
+__device__ __forceinline__ int window_expert(int raw, int lo, int E) {
+    const int64_t e = static_cast<int64_t>(raw) - lo;
+    return (e >= 0 && e < E) ? static_cast<int>(e) : -1;
+}
+
 __global__ void __launch_bounds__(kRouteThreads)
-route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int lo, int e_total,
                    int32_t* __restrict__ tile_counts, int stride, int32_t* __restrict__ token_of,
                    int64_t rmax, int32_t* err_flag) {
     extern __shared__ int32_t cnt[];  // [E]
@@ -89,11 +96,11 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
         if (i >= mine) break;
-        const int e = e_reg[i];
-        if (e < 0 || e >= E) {  // -1 is a masked pair (tk_tp_mask), anything else an error
-            if (e != -1) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
-            continue;
-        }
+        const int raw = e_reg[i];
+        // -1 is a masked pair (tk_tp_mask), an index outside [0, e_total) an error
+        if (raw != -1 && (raw < 0 || raw >= e_total)) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
+        const int e = window_expert(raw, lo, E);
+        if (e < 0) continue;
         atomicAdd(&cnt[e], 1);  // integer counts: the order of the additions does not matter
     }
     __syncthreads();
@@ -153,13 +160,14 @@ __device__ __forceinline__ void tile_scatter(const uint32_t* bitmap, const int32
     }
 }
 
-__device__ __forceinline__ void load_tile(const int32_t* topk_idx, int64_t p0, int n,
+// The tile's pairs' local experts (window_expert), this thread's share.
+__device__ __forceinline__ void load_tile(const int32_t* topk_idx, int64_t p0, int n, int lo, int E,
                                           int (&e_reg)[kPairsPerThread]) {
     const int mine = pairs_of_thread(n);
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
         if (i >= mine) break;
-        e_reg[i] = topk_idx[p0 + threadIdx.x + i * kRouteThreads];
+        e_reg[i] = window_expert(topk_idx[p0 + threadIdx.x + i * kRouteThreads], lo, E);
     }
 }
 
@@ -385,7 +393,7 @@ route_row_scan_kernel(int32_t* __restrict__ tile_counts, int stride, int E, int 
 // One CTA per tile: forms the expert offsets from counts itself (CTA 0 also writes them out),
 // then ranks and scatters the tile's pairs like the fused kernel.
 __global__ void __launch_bounds__(kRouteThreads)
-route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int align,
+route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int lo, int align,
                      const int32_t* __restrict__ tile_prefix, int stride,
                      const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                      int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
@@ -402,7 +410,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, 
     const int n = (min(T, t0 + kTileTokens) - t0) * k;
     const DivK divk(k);
     int e_reg[kPairsPerThread];
-    load_tile(topk_idx, p0, n, e_reg);
+    load_tile(topk_idx, p0, n, lo, E, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     __syncthreads();
     tile_mark(bitmap, e_reg, n, divk, E, err_flag);
@@ -421,7 +429,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, 
 // The scan and scatter of a count matrix too large for the fused kernel (and of every matrix
 // in the allocation-free entry point). With no tile the single-CTA scan writes the (zero)
 // counts and offsets.
-cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int k, int align,
+cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int k, int lo, int align,
                                      int32_t* tile_counts, int tiles, int stride, int32_t* counts,
                                      int32_t* offsets, int32_t* slot_of, int32_t* token_of,
                                      int32_t* err_flag, cudaStream_t s, const char** what) {
@@ -438,7 +446,7 @@ cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int 
     *what = "route_scatter_kernel";
     const size_t smem = static_cast<size_t>(E) * (kTileWords + 2) * sizeof(uint32_t);
     return launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
-                      T, E, k, align, static_cast<const int32_t*>(tile_counts), stride,
+                      T, E, k, lo, align, static_cast<const int32_t*>(tile_counts), stride,
                       static_cast<const int32_t*>(counts), offsets, slot_of, token_of, err_flag);
 }
 
@@ -447,7 +455,7 @@ cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int 
 // row's total for the offsets -- instead of waiting for a separate scan kernel. CTA 0 also
 // writes counts[] and offsets[]. The slot arithmetic is the same as route_scan + route_scatter.
 __global__ void __launch_bounds__(kRouteThreads, 1)
-route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int align,
+route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int lo, int align,
                           const int32_t* __restrict__ tile_counts, int stride,
                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                           int32_t* __restrict__ slot_of, int32_t* __restrict__ token_of,
@@ -465,7 +473,7 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
     const int n = (min(T, t0 + kTileTokens) - t0) * k;
     const DivK divk(k);
     int e_reg[kPairsPerThread];
-    load_tile(topk_idx, p0, n, e_reg);
+    load_tile(topk_idx, p0, n, lo, E, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     __syncthreads();
     // the tile's bitmap does not depend on the scan: marked before the row sums' loads (issuing
@@ -506,47 +514,73 @@ extern "C" size_t tk_route_map_workspace_bytes(int T, int E, int k) {
     return tk::route_map_workspace_bytes_impl(T, E);
 }
 
-extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int align,
-                                  int32_t* counts, int32_t* offsets, int32_t* slot_of,
-                                  int32_t* token_of, void* workspace, size_t workspace_bytes,
-                                  int32_t* err_flag, void* stream) {
-    using namespace tk;
-    if (T < 0) return fail_arg("tk_route_map: T=%d must be >= 0", T);
-    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("tk_route_map: E=%d outside [1, %d]", E, TK_MAX_EXPERTS);
-    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("tk_route_map: k=%d outside [1, %d]", k, TK_MAX_TOPK);
-    if (align < 1 || align > 4096) return fail_arg("tk_route_map: align=%d outside [1, 4096]", align);
+namespace tk {
+namespace {
+
+// The route map of the experts [lo, lo + E) of e_total (the whole map: lo = 0, E = e_total).
+tk_status route_map_impl(const char* fn, const int32_t* topk_idx, int T, int e_total, int k, int lo,
+                         int E, int align, int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                         int32_t* token_of, void* workspace, size_t workspace_bytes,
+                         int32_t* err_flag, void* stream) {
+    if (T < 0) return fail_arg("%s: T=%d must be >= 0", fn, T);
+    if (E < 1 || E > TK_MAX_EXPERTS) return fail_arg("%s: E=%d outside [1, %d]", fn, E, TK_MAX_EXPERTS);
+    if (lo < 0 || e_total < E || lo > e_total - E)
+        return fail_arg("%s: the window [%d, %d + %d) is not inside [0, %d)", fn, lo, lo, E, e_total);
+    if (k < 1 || k > TK_MAX_TOPK) return fail_arg("%s: k=%d outside [1, %d]", fn, k, TK_MAX_TOPK);
+    if (align < 1 || align > 4096) return fail_arg("%s: align=%d outside [1, 4096]", fn, align);
     const int64_t rmax = tk_max_rows(T, E, k, align);
-    if (rmax > INT32_MAX) return fail_arg("tk_route_map: T*k + E*(align-1) = %lld exceeds int32", (long long)rmax);
+    if (rmax > INT32_MAX) return fail_arg("%s: T*k + E*(align-1) = %lld exceeds int32", fn, (long long)rmax);
     if (counts == nullptr || offsets == nullptr || workspace == nullptr)
-        return fail_arg("tk_route_map: counts, offsets and workspace must not be NULL");
+        return fail_arg("%s: counts, offsets and workspace must not be NULL", fn);
     if (T > 0 && (topk_idx == nullptr || slot_of == nullptr))
-        return fail_arg("tk_route_map: topk_idx and slot_of must not be NULL");
-    if (rmax > 0 && token_of == nullptr) return fail_arg("tk_route_map: token_of must not be NULL");
+        return fail_arg("%s: topk_idx and slot_of must not be NULL", fn);
+    if (rmax > 0 && token_of == nullptr) return fail_arg("%s: token_of must not be NULL", fn);
     const size_t need = route_map_workspace_bytes_impl(T, E);
     if (workspace_bytes < need)
-        return fail_arg("tk_route_map: workspace holds %zu bytes, needs %zu", workspace_bytes, need);
+        return fail_arg("%s: workspace holds %zu bytes, needs %zu", fn, workspace_bytes, need);
     if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
-        return fail_arg("tk_route_map: workspace must be 16-byte aligned");
+        return fail_arg("%s: workspace must be 16-byte aligned", fn);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* tile_counts = static_cast<int32_t*>(workspace);
     const int tiles = num_tiles(T);
     const int stride = row_stride(tiles);
     const int count_grid = tiles > 0 ? tiles : 1;
     cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
-                                 static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
-                                 tile_counts, stride, token_of, rmax, err_flag);
+                                 static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k, lo,
+                                 e_total, tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
     if (tiles > 0 && static_cast<int64_t>(stride) * E <= kFusedMaxEntries) {
         const size_t smem = static_cast<size_t>(E) * (kTileWords + 3) * sizeof(uint32_t);
         err = launch_pdl(route_scan_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s,
-                         topk_idx, T, E, k, align, static_cast<const int32_t*>(tile_counts),
+                         topk_idx, T, E, k, lo, align, static_cast<const int32_t*>(tile_counts),
                          stride, counts, offsets, slot_of, token_of, err_flag);
         return check_launch(err, "route_scan_scatter_kernel");
     }
     const char* what = "";
-    err = launch_scan_then_scatter(topk_idx, T, E, k, align, tile_counts, tiles, stride, counts,
+    err = launch_scan_then_scatter(topk_idx, T, E, k, lo, align, tile_counts, tiles, stride, counts,
                                    offsets, slot_of, token_of, err_flag, s, &what);
     return check_launch(err, what);
+}
+
+}  // namespace
+}  // namespace tk
+
+extern "C" tk_status tk_route_map(const int32_t* topk_idx, int T, int E, int k, int align,
+                                  int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                                  int32_t* token_of, void* workspace, size_t workspace_bytes,
+                                  int32_t* err_flag, void* stream) {
+    return tk::route_map_impl("tk_route_map", topk_idx, T, E, k, 0, E, align, counts, offsets,
+                              slot_of, token_of, workspace, workspace_bytes, err_flag, stream);
+}
+
+extern "C" tk_status tk_route_map_window(const int32_t* topk_idx, int T, int E_total, int k,
+                                         int expert_lo, int E, int align, int32_t* counts,
+                                         int32_t* offsets, int32_t* slot_of, int32_t* token_of,
+                                         void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                                         void* stream) {
+    return tk::route_map_impl("tk_route_map_window", topk_idx, T, E_total, k, expert_lo, E, align,
+                              counts, offsets, slot_of, token_of, workspace, workspace_bytes,
+                              err_flag, stream);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -629,11 +663,11 @@ extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, 
     const int stride = row_stride(tiles);
     const int count_grid = tiles > 0 ? tiles : 1;
     cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
-                                 static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k,
-                                 tile_counts, stride, token_of, rmax, err_flag);
+                                 static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k, 0,
+                                 E, tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
     const char* what = "";
-    err = launch_scan_then_scatter(topk_idx, T, E, k, align, tile_counts, tiles, stride, counts,
+    err = launch_scan_then_scatter(topk_idx, T, E, k, 0, align, tile_counts, tiles, stride, counts,
                                    offsets, slot_of, token_of, err_flag, s, &what);
     return check_launch(err, what);
 }

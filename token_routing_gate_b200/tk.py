@@ -30,6 +30,7 @@ DEVERR_TIMEOUT = 16
 
 # every C entry point declared in include/tk_route.h
 ABI_SYMBOLS = ("tk_gate_topk", "tk_max_rows", "tk_route_map_workspace_bytes", "tk_route_map",
+               "tk_route_map_window",
                "tk_route_map_static", "tk_expand", "tk_reduce", "tk_reduce_masked", "tk_balance_stats_workspace_bytes",
                "tk_balance_stats", "tk_balance_score_sums", "tk_balance_finalize", "tk_tp_mask", "tk_reduce_backward_workspace_bytes",
                "tk_reduce_backward", "tk_expand_backward", "tk_ep_layout_workspace_bytes",
@@ -66,6 +67,8 @@ def _load():
     L.tk_route_map_workspace_bytes.restype = sz
     L.tk_route_map.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
     L.tk_route_map.restype = i32
+    L.tk_route_map_window.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.tk_route_map_window.restype = i32
     L.tk_route_map_static.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
     L.tk_route_map_static.restype = i32
     L.tk_expand.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
@@ -213,6 +216,28 @@ def route_map(topk_idx, E, align=1, out=None, err_flag=None, stream=None):
     _check("tk_route_map", lib.tk_route_map(
         _ptr(topk_idx, I32, T * k, "topk_idx"), T, E, k, align, _ptr(out.counts, I32, E, "counts"),
         _ptr(out.offsets, I32, E + 1, "offsets"), _ptr(out.slot_of, I32, T * k, "slot_of"),
+        _ptr(out.token_of, I32, max_rows(T, E, k, align), "token_of"),
+        _ws(out.workspace, route_map_workspace_bytes(T, E, k)), out.workspace.numel(), _flag(err_flag),
+        _stream(stream)))
+    return out
+
+
+def route_map_window(topk_idx, E_total, expert_lo, E, align=1, out=None, err_flag=None, stream=None):
+    """Route map of the experts [expert_lo, expert_lo + E) of E_total (others masked): the same
+    outputs as tp_mask followed by route_map with E experts, in one call."""
+    T, k = _shape2(topk_idx, "topk_idx")
+    dev = topk_idx.device
+    if out is None:
+        ws = max(route_map_workspace_bytes(T, E, k), 16)
+        out = RouteMap(torch.empty(E, dtype=torch.int32, device=dev),
+                       torch.empty(E + 1, dtype=torch.int32, device=dev),
+                       torch.empty(T, k, dtype=torch.int32, device=dev),
+                       torch.empty(max(max_rows(T, E, k, align), 1), dtype=torch.int32, device=dev),
+                       torch.empty((ws + 15) // 16, 16, dtype=torch.uint8, device=dev), align)
+    _check("tk_route_map_window", lib.tk_route_map_window(
+        _ptr(topk_idx, I32, T * k, "topk_idx"), T, E_total, k, expert_lo, E, align,
+        _ptr(out.counts, I32, E, "counts"), _ptr(out.offsets, I32, E + 1, "offsets"),
+        _ptr(out.slot_of, I32, T * k, "slot_of"),
         _ptr(out.token_of, I32, max_rows(T, E, k, align), "token_of"),
         _ws(out.workspace, route_map_workspace_bytes(T, E, k)), out.workspace.numel(), _flag(err_flag),
         _stream(stream)))
