@@ -70,6 +70,9 @@ __device__ __forceinline__ int window_expert(int raw, int lo, int E) {
     return (e >= 0 && e < E) ? static_cast<int>(e) : -1;
 }
 
+// kWindow: the experts [lo, lo + E) of e_total (tk_route_map_window); otherwise all E of them,
+// with the same code as before windows existed.
+template <bool kWindow>
 __global__ void __launch_bounds__(kRouteThreads)
 route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int lo, int e_total,
                    int32_t* __restrict__ tile_counts, int stride, int32_t* __restrict__ token_of,
@@ -96,11 +99,16 @@ route_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, in
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
         if (i >= mine) break;
-        const int raw = e_reg[i];
-        // -1 is a masked pair (tk_tp_mask), an index outside [0, e_total) an error
-        if (raw != -1 && (raw < 0 || raw >= e_total)) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
-        const int e = window_expert(raw, lo, E);
-        if (e < 0) continue;
+        int e = e_reg[i];
+        if constexpr (kWindow) {
+            // -1 is a masked pair (tk_tp_mask), an index outside [0, e_total) an error
+            if (e != -1 && (e < 0 || e >= e_total)) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
+            e = window_expert(e, lo, E);
+            if (e < 0) continue;
+        } else if (e < 0 || e >= E) {  // -1 is a masked pair (tk_tp_mask), anything else an error
+            if (e != -1) flag_error(err_flag, TK_DEVERR_EXPERT_RANGE);
+            continue;
+        }
         atomicAdd(&cnt[e], 1);  // integer counts: the order of the additions does not matter
     }
     __syncthreads();
@@ -160,14 +168,24 @@ __device__ __forceinline__ void tile_scatter(const uint32_t* bitmap, const int32
     }
 }
 
-// The tile's pairs' local experts (window_expert), this thread's share.
-__device__ __forceinline__ void load_tile(const int32_t* topk_idx, int64_t p0, int n, int lo, int E,
+__device__ __forceinline__ void load_tile(const int32_t* topk_idx, int64_t p0, int n,
                                           int (&e_reg)[kPairsPerThread]) {
     const int mine = pairs_of_thread(n);
 #pragma unroll
     for (int i = 0; i < kPairsPerThread; ++i) {
         if (i >= mine) break;
-        e_reg[i] = window_expert(topk_idx[p0 + threadIdx.x + i * kRouteThreads], lo, E);
+        e_reg[i] = topk_idx[p0 + threadIdx.x + i * kRouteThreads];
+    }
+}
+
+// The loaded indices as local experts (window_expert), in place. Called once the loads have
+// had the bitmap clearing and a barrier to arrive, so the mapping does not wait on them.
+__device__ __forceinline__ void to_window(int (&e_reg)[kPairsPerThread], int n, int lo, int E) {
+    const int mine = pairs_of_thread(n);
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        if (i >= mine) break;
+        e_reg[i] = window_expert(e_reg[i], lo, E);
     }
 }
 
@@ -392,6 +410,7 @@ route_row_scan_kernel(int32_t* __restrict__ tile_counts, int stride, int E, int 
 
 // One CTA per tile: forms the expert offsets from counts itself (CTA 0 also writes them out),
 // then ranks and scatters the tile's pairs like the fused kernel.
+template <bool kWindow>
 __global__ void __launch_bounds__(kRouteThreads)
 route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int lo, int align,
                      const int32_t* __restrict__ tile_prefix, int stride,
@@ -410,9 +429,10 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, 
     const int n = (min(T, t0 + kTileTokens) - t0) * k;
     const DivK divk(k);
     int e_reg[kPairsPerThread];
-    load_tile(topk_idx, p0, n, lo, E, e_reg);
+    load_tile(topk_idx, p0, n, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     __syncthreads();
+    if constexpr (kWindow) to_window(e_reg, n, lo, E);
     tile_mark(bitmap, e_reg, n, divk, E, err_flag);
     for (int e = threadIdx.x; e < E; e += kRouteThreads) total[e] = counts[e];
     __syncthreads();
@@ -429,6 +449,7 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, 
 // The scan and scatter of a count matrix too large for the fused kernel (and of every matrix
 // in the allocation-free entry point). With no tile the single-CTA scan writes the (zero)
 // counts and offsets.
+template <bool kWindow>
 cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int k, int lo, int align,
                                      int32_t* tile_counts, int tiles, int stride, int32_t* counts,
                                      int32_t* offsets, int32_t* slot_of, int32_t* token_of,
@@ -445,7 +466,7 @@ cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int 
     if (err != cudaSuccess) return err;
     *what = "route_scatter_kernel";
     const size_t smem = static_cast<size_t>(E) * (kTileWords + 2) * sizeof(uint32_t);
-    return launch_pdl(route_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
+    return launch_pdl(route_scatter_kernel<kWindow>, dim3(tiles), dim3(kRouteThreads), smem, s, topk_idx,
                       T, E, k, lo, align, static_cast<const int32_t*>(tile_counts), stride,
                       static_cast<const int32_t*>(counts), offsets, slot_of, token_of, err_flag);
 }
@@ -454,6 +475,7 @@ cudaError_t launch_scan_then_scatter(const int32_t* topk_idx, int T, int E, int 
 // CTA reads the whole (small) count matrix itself -- its own tile's prefix per expert, and every
 // row's total for the offsets -- instead of waiting for a separate scan kernel. CTA 0 also
 // writes counts[] and offsets[]. The slot arithmetic is the same as route_scan + route_scatter.
+template <bool kWindow>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int lo, int align,
                           const int32_t* __restrict__ tile_counts, int stride,
@@ -473,11 +495,12 @@ route_scan_scatter_kernel(const int32_t* __restrict__ topk_idx, int T, int E, in
     const int n = (min(T, t0 + kTileTokens) - t0) * k;
     const DivK divk(k);
     int e_reg[kPairsPerThread];
-    load_tile(topk_idx, p0, n, lo, E, e_reg);
+    load_tile(topk_idx, p0, n, e_reg);
     for (int i = threadIdx.x; i < E * kTileWords; i += kRouteThreads) bitmap[i] = 0u;
     __syncthreads();
     // the tile's bitmap does not depend on the scan: marked before the row sums' loads (issuing
     // those first, alongside the index loads, measured no faster)
+    if constexpr (kWindow) to_window(e_reg, n, lo, E);
     tile_mark(bitmap, e_reg, n, divk, E, err_flag);
     // per expert: the count over the tiles before this one, and the row total
     row_sums(tile_counts, stride, E, tile, before, total);
@@ -518,7 +541,8 @@ namespace tk {
 namespace {
 
 // The route map of the experts [lo, lo + E) of e_total (the whole map: lo = 0, E = e_total).
-tk_status route_map_impl(const char* fn, const int32_t* topk_idx, int T, int e_total, int k, int lo,
+template <bool kWindow>
+tk_status route_map_launch(const char* fn, const int32_t* topk_idx, int T, int e_total, int k, int lo,
                          int E, int align, int32_t* counts, int32_t* offsets, int32_t* slot_of,
                          int32_t* token_of, void* workspace, size_t workspace_bytes,
                          int32_t* err_flag, void* stream) {
@@ -545,21 +569,32 @@ tk_status route_map_impl(const char* fn, const int32_t* topk_idx, int T, int e_t
     const int tiles = num_tiles(T);
     const int stride = row_stride(tiles);
     const int count_grid = tiles > 0 ? tiles : 1;
-    cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
+    cudaError_t err = launch_pdl(route_count_kernel<kWindow>, dim3(count_grid), dim3(kRouteThreads),
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k, lo,
                                  e_total, tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
     if (tiles > 0 && static_cast<int64_t>(stride) * E <= kFusedMaxEntries) {
         const size_t smem = static_cast<size_t>(E) * (kTileWords + 3) * sizeof(uint32_t);
-        err = launch_pdl(route_scan_scatter_kernel, dim3(tiles), dim3(kRouteThreads), smem, s,
+        err = launch_pdl(route_scan_scatter_kernel<kWindow>, dim3(tiles), dim3(kRouteThreads), smem, s,
                          topk_idx, T, E, k, lo, align, static_cast<const int32_t*>(tile_counts),
                          stride, counts, offsets, slot_of, token_of, err_flag);
         return check_launch(err, "route_scan_scatter_kernel");
     }
     const char* what = "";
-    err = launch_scan_then_scatter(topk_idx, T, E, k, lo, align, tile_counts, tiles, stride, counts,
-                                   offsets, slot_of, token_of, err_flag, s, &what);
+    err = launch_scan_then_scatter<kWindow>(topk_idx, T, E, k, lo, align, tile_counts, tiles, stride,
+                                            counts, offsets, slot_of, token_of, err_flag, s, &what);
     return check_launch(err, what);
+}
+
+tk_status route_map_impl(const char* fn, const int32_t* topk_idx, int T, int e_total, int k, int lo,
+                         int E, int align, int32_t* counts, int32_t* offsets, int32_t* slot_of,
+                         int32_t* token_of, void* workspace, size_t workspace_bytes,
+                         int32_t* err_flag, void* stream) {
+    if (lo == 0 && E == e_total)
+        return route_map_launch<false>(fn, topk_idx, T, e_total, k, lo, E, align, counts, offsets,
+                                       slot_of, token_of, workspace, workspace_bytes, err_flag, stream);
+    return route_map_launch<true>(fn, topk_idx, T, e_total, k, lo, E, align, counts, offsets, slot_of,
+                                  token_of, workspace, workspace_bytes, err_flag, stream);
 }
 
 }  // namespace
@@ -662,12 +697,12 @@ extern "C" tk_status tk_route_map_static(const int32_t* topk_idx, int T, int E, 
     const int tiles = num_tiles(T);
     const int stride = row_stride(tiles);
     const int count_grid = tiles > 0 ? tiles : 1;
-    cudaError_t err = launch_pdl(route_count_kernel, dim3(count_grid), dim3(kRouteThreads),
+    cudaError_t err = launch_pdl(route_count_kernel<false>, dim3(count_grid), dim3(kRouteThreads),
                                  static_cast<size_t>(E) * sizeof(int32_t), s, topk_idx, T, E, k, 0,
                                  E, tile_counts, stride, token_of, rmax, err_flag);
     if (err != cudaSuccess) return check_launch(err, "route_count_kernel");
     const char* what = "";
-    err = launch_scan_then_scatter(topk_idx, T, E, k, 0, align, tile_counts, tiles, stride, counts,
-                                   offsets, slot_of, token_of, err_flag, s, &what);
+    err = launch_scan_then_scatter<false>(topk_idx, T, E, k, 0, align, tile_counts, tiles, stride,
+                                          counts, offsets, slot_of, token_of, err_flag, s, &what);
     return check_launch(err, what);
 }
