@@ -122,7 +122,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // 1-D bulk copy global -> shared (TMA engine), completion counted on `bar` in bytes.
-// No multicast. dst/src 16-byte aligned, bytes a multiple of 16.
+// One destination CTA (no cluster broadcast). dst/src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
                                           uint64_t* bar) {
     asm volatile(
